@@ -1,0 +1,214 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module draws random numbers and lays out tables; it holds none of the
+attention arithmetic and none of the row-write addressing.  Both the oracle
+and the CUDA path receive what it returns:
+
+  * the oracle gets per-stream LINEAR caches ``[len_s][Hkv][d]`` and the query
+    rows;
+  * the CUDA path gets the same rows and writes them into its pages itself
+    (through its own row write), guided by the page table built here.
+
+Values are drawn as float32 from numpy's PCG64 (one independent SeedSequence
+per stream and tensor, so one stream can be regenerated alone for sampled
+checks at full size) and rounded to bf16 with round-to-nearest-even.  bf16 is
+handled as raw ``uint16`` bit patterns everywhere.
+
+Workloads (synthetic stand-ins for the pages' served runs):
+  * ``parity_small``   one stream, 1 KV head, GQA 4, d 128, 1,037 positions in
+    pages of 512 (last one partial) in a pool of 8, one decode row;
+  * ``decode_12x40k``  12 streams at 40,960, 8 KV / 32 query heads, d 128,
+    pool 1.2x the pages needed, one row per stream (TensorFold #1620's
+    ``--parallel 12 --context 40960`` cells);
+  * ``verify_4x131k``  4 streams at 131,072, 4 KV / 32 query heads (GQA 8),
+    d 128, 8-row causal windows (TensorFold #2730: eight rows, 131,072 context,
+    four streams);
+  * ``hd512_verify``   16 streams, lengths uniform in [2,048, 9,216], 2 KV / 16
+    query heads, d 512, 4-row windows, K/V ~ N(0, 0.5^2) (TensorFold #1620's
+    head dim 512 global layer, four-row cells);
+  * ``prompt_9216``    one 9,216-token prompt written into shuffled pages, then
+    attended in causal chunks of 512 rows, 8 KV / 32 query heads, d 128.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+BF16_NAN = np.uint16(0x7FC0)
+
+
+def bf16_from_f32(x) -> np.ndarray:
+    """Round float32 values to bf16 (round to nearest, ties to even); returns uint16 bits."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    out = rounded.astype(np.uint16)
+    nan = np.isnan(x)
+    if nan.any():
+        out[nan] = BF16_NAN
+    return out
+
+
+def f32_from_bf16(b) -> np.ndarray:
+    """Widen bf16 bit patterns to float32 (exact)."""
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def _rng(*key: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(k) for k in key])))
+
+
+def normal_bf16(key, shape, sigma: float = 1.0) -> np.ndarray:
+    """bf16 bits of N(0, sigma^2) samples of the given shape, seeded by the int tuple ``key``."""
+    x = _rng(*key).standard_normal(size=shape, dtype=np.float32)
+    if sigma != 1.0:
+        x *= np.float32(sigma)
+    return bf16_from_f32(x)
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    n_streams: int
+    n_kv_heads: int
+    group: int                 # query heads per KV head
+    head_dim: int
+    page_size: int
+    rows: int                  # window rows W (decode 1, verify <= 8, prompt chunk)
+    seed: int
+    kv_sigma: float = 1.0
+    q_sigma: float = 1.0
+    lens: tuple = ()           # fixed per-stream lengths, or () with len_range
+    len_range: tuple = ()      # (lo, hi) inclusive uniform integer lengths
+    pool_factor: float = 1.2
+    n_pages: int = 0           # fixed pool size (0: ceil(pool_factor * needed) + 1)
+    prompt_len: int = 0        # >0: one prompt attended in chunks of ``rows``
+
+    @property
+    def n_q_heads(self) -> int:
+        return self.n_kv_heads * self.group
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+
+WORKLOADS = {
+    "parity_small": Workload("parity_small", 1, 1, 4, 128, 512, 1, seed=1, lens=(1037,),
+                             n_pages=8),
+    "decode_12x40k": Workload("decode_12x40k", 12, 8, 4, 128, 512, 1, seed=2,
+                              lens=(40960,) * 12),
+    "verify_4x131k": Workload("verify_4x131k", 4, 4, 8, 128, 512, 8, seed=3,
+                              lens=(131072,) * 4),
+    "hd512_verify": Workload("hd512_verify", 16, 2, 8, 512, 512, 4, seed=4, kv_sigma=0.5,
+                             len_range=(2048, 9216)),
+    "prompt_9216": Workload("prompt_9216", 1, 8, 4, 128, 512, 512, seed=5, lens=(9216,),
+                            prompt_len=9216),
+}
+
+
+def stream_lens(w: Workload) -> np.ndarray:
+    if w.lens:
+        return np.array(w.lens, dtype=np.int32)
+    lo, hi = w.len_range
+    return _rng(w.seed, 0).integers(lo, hi + 1, size=w.n_streams).astype(np.int32)
+
+
+def pages_needed(lens, page_size: int) -> np.ndarray:
+    return (np.asarray(lens, dtype=np.int64) + page_size - 1) // page_size
+
+
+def page_table(w: Workload, lens, spare_fill: bool = True):
+    """Seeded shuffled page table.
+
+    Returns (table int32 [S][stride], n_pages, spare_ids).  Stream s owns
+    ``ceil(len_s / P)`` distinct pool pages drawn from one seeded permutation
+    of the pool; entries past a stream's pages point at spare (NaN-filled)
+    pages, so a kernel that reads past a stream's end would read NaN.
+    """
+    P = w.page_size
+    need = pages_needed(lens, P)
+    stride = int(need.max())
+    total = int(need.sum())
+    n_pages = w.n_pages or int(math.ceil(w.pool_factor * total)) + 1
+    assert n_pages > total, "the pool needs at least one spare page"
+    perm = _rng(w.seed, 7).permutation(n_pages).astype(np.int32)
+    spare = perm[total:]
+    table = np.empty((len(lens), stride), dtype=np.int32)
+    off = 0
+    for s, n in enumerate(need):
+        table[s, :n] = perm[off:off + n]
+        table[s, n:] = spare[(s + np.arange(stride - n)) % len(spare)] if spare_fill else -1
+        off += n
+    return table, n_pages, spare
+
+
+def identity_table(lens, page_size: int):
+    """Pages laid out in order: stream 0's pages first, then stream 1's, ... (no shuffle)."""
+    need = pages_needed(lens, page_size)
+    stride = int(need.max())
+    total = int(need.sum())
+    table = np.full((len(lens), stride), total, dtype=np.int32)   # page `total` is the spare
+    off = 0
+    for s, n in enumerate(need):
+        table[s, :n] = np.arange(off, off + n, dtype=np.int32)
+        off += n
+    return table, total + 1
+
+
+def kv_rows(w: Workload, s: int, length: int):
+    """Linear K and V of stream s: two uint16 arrays [length][Hkv][d] (bf16 bits)."""
+    shape = (length, w.n_kv_heads, w.head_dim)
+    return (normal_bf16((w.seed, 1, s), shape, w.kv_sigma),
+            normal_bf16((w.seed, 2, s), shape, w.kv_sigma))
+
+
+def q_rows(w: Workload, rows: int | None = None, tag: int = 0):
+    """Query rows [S][W][Hq][d] (bf16 bits)."""
+    W = w.rows if rows is None else rows
+    return normal_bf16((w.seed, 3, tag), (w.n_streams, W, w.n_q_heads, w.head_dim), w.q_sigma)
+
+
+@dataclasses.dataclass
+class Case:
+    """One attention call's inputs, in both views."""
+    w: Workload
+    lens: np.ndarray            # int32 [S], positions after this step's rows
+    rows: int                   # W
+    q: np.ndarray               # uint16 [S][W][Hq][d]
+    k_lin: list                 # S x uint16 [len_s][Hkv][d]
+    v_lin: list
+    table: np.ndarray           # int32 [S][stride]
+    n_pages: int
+
+    @property
+    def new_k(self) -> np.ndarray:
+        """This step's rows [S][W][Hkv][d]: the last W positions of each stream."""
+        return np.stack([k[len(k) - self.rows:] for k in self.k_lin])
+
+    @property
+    def new_v(self) -> np.ndarray:
+        return np.stack([v[len(v) - self.rows:] for v in self.v_lin])
+
+
+def make_case(w: Workload, lens=None, rows: int | None = None, table=None, n_pages=None,
+              streams=None) -> Case:
+    """Build a call's inputs.  ``streams`` restricts K/V generation to some streams
+    (others get empty caches; for sampled checks at full size)."""
+    lens = stream_lens(w) if lens is None else np.asarray(lens, dtype=np.int32)
+    W = w.rows if rows is None else rows
+    if table is None:
+        table, n_pages, _ = page_table(w, lens)
+    k_lin, v_lin = [], []
+    for s in range(len(lens)):
+        if streams is None or s in streams:
+            k, v = kv_rows(w, s, int(lens[s]))
+        else:
+            k = v = np.zeros((0, w.n_kv_heads, w.head_dim), dtype=np.uint16)
+        k_lin.append(k)
+        v_lin.append(v)
+    wq = dataclasses.replace(w, n_streams=len(lens))
+    return Case(w, lens, W, q_rows(wq, W), k_lin, v_lin, table, n_pages)

@@ -1,0 +1,215 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+Each ``pin_*`` function takes an optional compiled oracle library (``lib``) so
+the same checks can be run against copies of the oracle with a planted
+mistake (see test_oracle_planted.py).  A pin raises AssertionError (or the
+oracle's ValueError) when it fails.
+
+What pins what:
+  * hand-derived worked examples (tests/golden/hand_examples.json): exact
+    fractions for two keys, a two-row causal window, grouped heads;
+  * brute force on tiny inputs: a separate pure-Python formulation (full
+    score matrix, explicit mask, no max subtraction, math.fsum);
+  * a library routine: torch's scaled_dot_product_attention in fp64 with its
+    grouped-query option and an explicit window mask;
+  * closed forms: constant values, one visible key, zero query, a dominant
+    key;
+  * invariants: causality, verify row == decode at that position, thread
+    count does not change a bit;
+  * the row write: per-element brute force on a tiny pool, untouched bytes.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _bf(x):
+    return synth.bf16_from_f32(np.asarray(x, dtype=np.float32))
+
+
+def _f64(b):
+    return synth.f32_from_bf16(b).astype(np.float64)
+
+
+def _random_case(rng, S, W, Hkv, G, d, lens, sigma=1.0):
+    q = _bf(rng.standard_normal((S, W, Hkv * G, d)))
+    k = [_bf(sigma * rng.standard_normal((n, Hkv, d))) for n in lens]
+    v = [_bf(sigma * rng.standard_normal((n, Hkv, d))) for n in lens]
+    return q, k, v
+
+
+def pin_hand_examples(lib=None):
+    with open(os.path.join(GOLDEN, "hand_examples.json")) as f:
+        data = json.load(f)
+    scales = {"ln2": math.log(2.0), "ln3": math.log(3.0), "1": 1.0}
+    for ex in data["examples"]:
+        q = _bf(ex["q"])
+        k = [_bf(x) for x in ex["k"]]
+        v = [_bf(x) for x in ex["v"]]
+        out = oracle.attend(q, k, v, ex["lens"], ex["W"], ex["G"], scales[ex["scale"]], lib=lib)
+        np.testing.assert_allclose(out, np.array(ex["out"]), rtol=0, atol=1e-13,
+                                   err_msg=ex["name"])
+
+
+def brute_force(q, k, v, lens, W, G, scale):
+    """Pure-Python attention: full score matrix, explicit mask, no max shift."""
+    S, _, Hq, d = q.shape
+    qf = _f64(q)
+    out = np.zeros(q.shape, dtype=np.float64)
+    for s in range(S):
+        kf, vf = _f64(k[s]), _f64(v[s])
+        n = lens[s]
+        for r in range(W):
+            for h in range(Hq):
+                g = h // G
+                e = []
+                for j in range(n):
+                    visible = j <= n - W + r
+                    if visible:
+                        x = scale * math.fsum(qf[s, r, h, i] * kf[j, g, i] for i in range(d))
+                        e.append((j, math.exp(x)))
+                z = math.fsum(w for _, w in e)
+                for i in range(d):
+                    out[s, r, h, i] = math.fsum(w * vf[j, g, i] for j, w in e) / z
+    return out
+
+
+def pin_brute_force(lib=None):
+    rng = np.random.default_rng(11)
+    for (S, W, Hkv, G, d, lens) in [(1, 1, 1, 1, 4, [1]), (2, 3, 2, 2, 4, [3, 6]),
+                                    (2, 2, 1, 4, 8, [5, 2]), (1, 3, 2, 1, 3, [4])]:
+        q, k, v = _random_case(rng, S, W, Hkv, G, d, lens)
+        scale = 1.0 / math.sqrt(d)
+        got = oracle.attend(q, k, v, lens, W, G, scale, lib=lib)
+        want = brute_force(q, k, v, lens, W, G, scale)
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def pin_sdpa(lib=None):
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(12)
+    for (S, W, Hkv, G, d, lens) in [(3, 4, 2, 4, 16, [4, 37, 9]), (2, 8, 1, 8, 32, [8, 70]),
+                                    (1, 1, 3, 2, 8, [50])]:
+        q, k, v = _random_case(rng, S, W, Hkv, G, d, lens)
+        scale = 1.0 / math.sqrt(d)
+        got = oracle.attend(q, k, v, lens, W, G, scale, lib=lib)
+        for s in range(S):
+            n = lens[s]
+            qt = torch.from_numpy(_f64(q[s])).permute(1, 0, 2)[None]          # [1,Hq,W,d]
+            kt = torch.from_numpy(_f64(k[s])).permute(1, 0, 2)[None]          # [1,Hkv,n,d]
+            vt = torch.from_numpy(_f64(v[s])).permute(1, 0, 2)[None]
+            pos = torch.arange(n)[None, :]
+            rowpos = (n - W + torch.arange(W))[:, None]
+            mask = pos <= rowpos                                              # [W, n]
+            ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale,
+                                                 enable_gqa=True)
+            np.testing.assert_allclose(got[s], ref[0].permute(1, 0, 2).numpy(), rtol=0,
+                                       atol=1e-12)
+
+
+def pin_closed_forms(lib=None):
+    rng = np.random.default_rng(13)
+    S, W, Hkv, G, d = 2, 3, 2, 4, 16
+    lens = [7, 3]
+    q, k, v = _random_case(rng, S, W, Hkv, G, d, lens)
+    scale = 1.0 / math.sqrt(d)
+    # constant values: the output is that constant whatever the weights
+    vc = [np.full_like(x, _bf([1.5])[0]) for x in v]
+    out = oracle.attend(q, k, vc, lens, W, G, scale, lib=lib)
+    np.testing.assert_allclose(out, 1.5, rtol=0, atol=1e-14)
+    # one visible key (len == W == 1): the output is that key's value
+    q1, k1, v1 = _random_case(rng, 2, 1, Hkv, G, d, [1, 1])
+    out = oracle.attend(q1, k1, v1, [1, 1], 1, G, scale, lib=lib)
+    for s in range(2):
+        for h in range(Hkv * G):
+            np.testing.assert_allclose(out[s, 0, h], _f64(v1[s][0, h // G]), rtol=0, atol=0)
+    # zero query: uniform weights, the output is the mean of the visible values
+    q0 = np.zeros_like(q)
+    out = oracle.attend(q0, k, v, lens, W, G, scale, lib=lib)
+    for s in range(S):
+        for r in range(W):
+            t = lens[s] - W + r
+            for h in range(Hkv * G):
+                want = _f64(v[s][: t + 1, h // G]).mean(axis=0)
+                np.testing.assert_allclose(out[s, r, h], want, rtol=0, atol=1e-13)
+    # a dominant key: one visible key's score sits 40 above the rest -> its value
+    d2 = 8
+    n = 6
+    qd = np.zeros((1, 1, 1, d2), dtype=np.uint16)
+    qd[0, 0, 0, 0] = _bf([1.0])[0]
+    kd = np.zeros((n, 1, d2), dtype=np.uint16)
+    kd[3, 0, 0] = _bf([40.0])[0]
+    vd = _bf(rng.standard_normal((n, 1, d2)))
+    out = oracle.attend(qd, [kd], [vd], [n], 1, 1, 1.0, lib=lib)
+    np.testing.assert_allclose(out[0, 0, 0], _f64(vd[3, 0]), rtol=0, atol=1e-15 + 12 * math.exp(-40) * 8)
+
+
+def pin_invariants(lib=None):
+    rng = np.random.default_rng(14)
+    S, W, Hkv, G, d = 2, 4, 2, 2, 16
+    lens = [9, 20]
+    q, k, v = _random_case(rng, S, W, Hkv, G, d, lens)
+    scale = 0.25
+    base = oracle.attend(q, k, v, lens, W, G, scale, lib=lib)
+    # causality: changing K/V at positions after row r leaves row r unchanged, and
+    # changing the position of row r itself changes it
+    for s in range(S):
+        for r in range(W):
+            t = lens[s] - W + r
+            k2 = [x.copy() for x in k]
+            v2 = [x.copy() for x in v]
+            k2[s][t + 1:] = _bf(rng.standard_normal(k2[s][t + 1:].shape))
+            v2[s][t + 1:] = _bf(rng.standard_normal(v2[s][t + 1:].shape))
+            out = oracle.attend(q, k2, v2, lens, W, G, scale, lib=lib)
+            np.testing.assert_array_equal(out[s, r], base[s, r])
+            v3 = [x.copy() for x in v]
+            v3[s][t] = _bf(_f64(v3[s][t]) + 3.0)
+            out = oracle.attend(q, k, v3, lens, W, G, scale, lib=lib)
+            assert np.abs(out[s, r] - base[s, r]).max() > 1e-6
+    # verify row r == decode of that row alone with len' = len - W + r + 1
+    for r in range(W):
+        lens_r = [n - W + r + 1 for n in lens]
+        out = oracle.attend(q[:, r:r + 1].copy(), [x[:n] for x, n in zip(k, lens_r)],
+                            [x[:n] for x, n in zip(v, lens_r)], lens_r, 1, G, scale, lib=lib)
+        np.testing.assert_allclose(out[:, 0], base[:, r], rtol=0, atol=1e-14)
+    # the thread count changes no bit
+    out4 = oracle.attend(q, k, v, lens, W, G, scale, threads=4, lib=lib)
+    np.testing.assert_array_equal(out4, base)
+
+
+def pin_put_rows(lib=None):
+    rng = np.random.default_rng(15)
+    n_pages, Hkv, P, d = 7, 2, 4, 3
+    lens = np.array([6, 9], dtype=np.int32)
+    W = 3
+    table = np.array([[5, 1, 6], [0, 3, 2]], dtype=np.int32)
+    kp = np.full((n_pages, Hkv, P, d), synth.BF16_NAN, dtype=np.uint16)
+    vp = kp.copy()
+    kr = rng.integers(0, 0x7F00, size=(2, W, Hkv, d)).astype(np.uint16)
+    vr = rng.integers(0, 0x7F00, size=(2, W, Hkv, d)).astype(np.uint16)
+    oracle.put_rows(kp, vp, table, lens, kr, vr, lib=lib)
+    want_k = np.full_like(kp, synth.BF16_NAN)
+    want_v = want_k.copy()
+    for s in range(2):
+        for r in range(W):
+            pos = int(lens[s]) - W + r
+            for h in range(Hkv):
+                for i in range(d):
+                    want_k[table[s][pos // P], h, pos % P, i] = kr[s, r, h, i]
+                    want_v[table[s][pos // P], h, pos % P, i] = vr[s, r, h, i]
+    np.testing.assert_array_equal(kp, want_k)
+    np.testing.assert_array_equal(vp, want_v)
+
+
+ALL_PINS = [pin_hand_examples, pin_brute_force, pin_sdpa, pin_closed_forms, pin_invariants,
+            pin_put_rows]
