@@ -1,0 +1,164 @@
+/*
+ * tf_paged.h -- attention over a paged KV cache on NVIDIA B200 (sm_100a).
+ *
+ * Keys and values live in fixed pages of `page_size` positions drawn from
+ * one shared pool; every stream reads its positions through its own row of
+ * a page table.  The library provides the row write that copies new K/V rows
+ * into their pages, and grouped-query attention for single-row decode,
+ * draft-verify windows (causal inside the window) and chunked prompt rows.
+ *
+ * Sources (the TensorFold pull-request pages this library follows):
+ *  - TensorFold #1620, "Kolibri-1's full layers take their K/V from pages of
+ *    the core pool", opening comment:
+ *      * "Pages of 512 positions": the pool and its fixed page size;
+ *      * "Writes": new K/V rows are copied into the pages (tf_kv_put_rows);
+ *      * "Reads": prompt rows, decode and drafted verify read keys through a
+ *        page table given in the call's stream order (the tf_paged_attn_*
+ *        calls);
+ *    and its later comment on per-tile page lookup: a tile's page is looked
+ *    up once per tile, and paging leaves the result bits unchanged.
+ *  - TensorFold #2730, "an eight-row verify window", section "What this
+ *    changes": a verify window is the pending token plus up to seven drafts.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  Layouts (all row-major, element counts, no padding):
+ *    K pool, V pool  bf16  [n_pages][n_kv_heads][page_size][head_dim]  device
+ *    table           int32 [n_streams][table_stride]                   device
+ *    lens            int32 [n_streams]                                  device
+ *    q               bf16  [n_streams][rows][n_q_heads][head_dim]       device
+ *    out             fp32  [n_streams][rows][n_q_heads][head_dim]       device
+ *    k_rows, v_rows  bf16  [n_streams][rows][n_kv_heads][head_dim]      device
+ *
+ *  lens[s] counts the positions of stream s AFTER this step's rows are
+ *  written.  Window row r (0 <= r < rows) sits at position
+ *  lens[s] - rows + r and attends to positions 0 .. lens[s] - rows + r.
+ *  Position j of stream s lives in pool page table[s][j / page_size], slot
+ *  j % page_size.  Query head h reads KV head h / (n_q_heads / n_kv_heads).
+ *
+ *  The output is softmax(scale * q . k) weighted sum of v, accumulated in
+ *  fp32 from bf16 inputs.  Which pool pages hold a stream's positions never
+ *  changes a bit of the result: the arithmetic depends only on positions,
+ *  lens, rows and the host arguments.
+ *
+ *  Ownership: the caller owns every buffer.  The library allocates nothing
+ *  and keeps no state between calls; each call enqueues kernels on the
+ *  caller's CUDA stream (`stream` is a cudaStream_t; NULL is the legacy
+ *  default stream) and returns without waiting.
+ *
+ *  Errors: every call checks its host arguments before enqueueing anything
+ *  and returns a TF_* status; on a non-zero status nothing was enqueued
+ *  (TF_ECUDA: a launch failed).  lens and table are device data and are
+ *  checked on the device: a stream whose length is outside
+ *  [rows, min(max_len, table_stride * page_size)] is skipped and its
+ *  outputs are set to NaN; a page id outside [0, n_pages) is never read.
+ *  Such events set bits in the workspace's status word (tf_workspace_status).
+ *  Table entries past ceil(lens[s] / page_size) are never read, and pool
+ *  slots at or past lens[s] never reach an output, whatever they hold.
+ *
+ *  Graph capture: lens and table are read on the device, and max_len only
+ *  bounds the launch, so one captured graph serves growing lengths up to
+ *  max_len.
+ */
+#ifndef TF_PAGED_H
+#define TF_PAGED_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TF_API __attribute__((visibility("default")))
+#else
+#define TF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every call. */
+#define TF_OK 0
+#define TF_EINVAL 1        /* a NULL pointer, a bad size or an inconsistent shape */
+#define TF_EUNSUPPORTED 2  /* a shape this build has no kernel for (head_dim, page_size) */
+#define TF_ENOSPACE 3      /* the workspace is smaller than tf_paged_attn_workspace_bytes */
+#define TF_ECUDA 4         /* a CUDA launch or query failed */
+
+/* Bits of the device-side status word (tf_workspace_status). */
+#define TF_DEV_BAD_LEN 1u   /* some lens[s] outside [rows, min(max_len, table_stride*page_size)] */
+#define TF_DEV_BAD_PAGE 2u  /* some table entry in use outside [0, n_pages) */
+#define TF_DEV_TIMEOUT 4u   /* a pipeline wait gave up (an internal error) */
+
+/* The pool: K and V pages, device memory, 16-byte aligned.
+ * page_size must be a multiple of 64; head_dim must be 128 or 512. */
+typedef struct tf_kv_pool {
+    void *k_pool;
+    void *v_pool;
+    int32_t n_pages;
+    int32_t n_kv_heads;
+    int32_t page_size;
+    int32_t head_dim;
+} tf_kv_pool;
+
+/* The streams of one call: page table, lengths (device) and a host upper
+ * bound on the lengths.  max_len <= table_stride * page_size. */
+typedef struct tf_streams {
+    const int32_t *table;
+    int32_t table_stride;
+    const int32_t *lens;
+    int32_t n_streams;
+    int32_t max_len;
+} tf_streams;
+
+/* Row write (TensorFold #1620, opening comment, "Writes").
+ * Copies `rows` new K and V rows per stream into their pages: row r of
+ * stream s (k_rows[s][r][kh][:]) goes to position lens[s] - rows + r.  The
+ * copy is bitwise; nothing else in the pool is touched.  A row whose
+ * stream length or page id is out of range is skipped.  rows >= 1. */
+TF_API int tf_kv_put_rows(const tf_kv_pool *pool, const tf_streams *streams,
+                   const void *k_rows, const void *v_rows, int32_t rows,
+                   void *stream);
+
+/* Workspace bytes an attention call with these arguments needs (0 on a bad
+ * argument).  The workspace holds split-context partial results and the
+ * status word; it needs no initialisation and may be reused by later calls
+ * on the same stream. */
+TF_API size_t tf_paged_attn_workspace_bytes(const tf_kv_pool *pool,
+                                     const tf_streams *streams,
+                                     int32_t n_q_heads, int32_t rows);
+
+/* Single-row decode (TensorFold #1620, opening comment, "Reads": decode).
+ * Same as tf_paged_attn_verify with rows = 1. */
+TF_API int tf_paged_attn_decode(const tf_kv_pool *pool, const tf_streams *streams,
+                         const void *q, int32_t n_q_heads, float scale,
+                         float *out, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* Draft-verify window (TensorFold #1620 "Reads": drafted verify; TensorFold
+ * #2730 "What this changes": the pending token plus up to seven drafts).
+ * rows in [1, 8]; row r sees positions 0 .. lens[s] - rows + r. */
+TF_API int tf_paged_attn_verify(const tf_kv_pool *pool, const tf_streams *streams,
+                         const void *q, int32_t n_q_heads, int32_t rows,
+                         float scale, float *out, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Chunked prompt rows (TensorFold #1620 "Reads": prompts through the paged
+ * prompt kernels).  The same causal rule as verify for a chunk of
+ * rows in [1, 4096] positions: the chunk is the last `rows` positions. */
+TF_API int tf_paged_attn_prompt(const tf_kv_pool *pool, const tf_streams *streams,
+                         const void *q, int32_t n_q_heads, int32_t rows,
+                         float scale, float *out, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Reads the workspace's device status word (TF_DEV_* bits accumulated by
+ * the attention calls since the last read) into *flags and clears it.
+ * Synchronises `stream`.  Returns TF_OK, TF_EINVAL or TF_ECUDA. */
+TF_API int tf_workspace_status(void *workspace, uint32_t *flags, void *stream);
+
+/* A static, human-readable name for a status code. */
+TF_API const char *tf_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TF_PAGED_H */

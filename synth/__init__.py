@@ -51,6 +51,31 @@ def bf16_from_f32(x) -> np.ndarray:
     return out
 
 
+def _seed_int(*key: int) -> int:
+    """A 63-bit seed for torch's generator, mixed from an int tuple."""
+    return int(np.random.SeedSequence([int(k) for k in key]).generate_state(2, np.uint64)[0]
+               >> np.uint64(1))
+
+
+def normal_bf16_torch(key, shape, sigma: float = 1.0, device="cuda"):
+    """Like normal_bf16 but drawn by torch's generator on ``device`` (fast for the
+    full-size workloads); a different stream of numbers than the numpy one.
+    Returns a torch.bfloat16 tensor (rounded to nearest even by torch)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(_seed_int(*key))
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if sigma != 1.0:
+        x.mul_(sigma)
+    return x.to(torch.bfloat16)
+
+
+def to_bits(t) -> np.ndarray:
+    """bf16 torch tensor -> host uint16 bit patterns."""
+    import torch
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
 def f32_from_bf16(b) -> np.ndarray:
     """Widen bf16 bit patterns to float32 (exact)."""
     b = np.ascontiguousarray(b, dtype=np.uint16)
@@ -164,6 +189,19 @@ def kv_rows(w: Workload, s: int, length: int):
     shape = (length, w.n_kv_heads, w.head_dim)
     return (normal_bf16((w.seed, 1, s), shape, w.kv_sigma),
             normal_bf16((w.seed, 2, s), shape, w.kv_sigma))
+
+
+def kv_rows_torch(w: Workload, s: int, length: int, device="cuda"):
+    """Linear K and V of stream s drawn on the device: two bf16 tensors [length][Hkv][d]."""
+    shape = (length, w.n_kv_heads, w.head_dim)
+    return (normal_bf16_torch((w.seed, 11, s), shape, w.kv_sigma, device),
+            normal_bf16_torch((w.seed, 12, s), shape, w.kv_sigma, device))
+
+
+def q_rows_torch(w: Workload, n_streams: int, rows: int, tag: int = 0, device="cuda"):
+    """Query rows [S][W][Hq][d] drawn on the device (bf16 tensor)."""
+    return normal_bf16_torch((w.seed, 13, tag), (n_streams, rows, w.n_q_heads, w.head_dim),
+                             w.q_sigma, device)
 
 
 def q_rows(w: Workload, rows: int | None = None, tag: int = 0):

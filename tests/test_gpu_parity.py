@@ -1,0 +1,151 @@
+"""The CUDA path against the fp64 oracle, and its byte-level guarantees (B200)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_cases import TOL, DeviceCase, bf16_tensor, max_abs, nan_pool
+
+pytestmark = pytest.mark.gpu
+
+
+def small_workload(d, G, P, W, Hkv=2, seed=100, sigma=1.0):
+    return synth.Workload("sweep", 0, Hkv, G, d, P, W, seed=seed, kv_sigma=sigma)
+
+
+def run_parity(w, lens, rows, table=None, n_pages=None):
+    case = synth.make_case(w, lens=lens, rows=rows, table=table, n_pages=n_pages)
+    dc = DeviceCase(case)
+    out = dc.attend()
+    torch.cuda.synchronize()
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, rows, w.group, w.scale,
+                        threads=8)
+    assert torch.isfinite(out).all()
+    err = max_abs(out, ref)
+    assert err <= TOL, err
+    return case, dc, out
+
+
+def test_parity_small_workload():
+    w = synth.WORKLOADS["parity_small"]
+    run_parity(w, None, 1)
+
+
+@pytest.mark.parametrize("d", [128, 512])
+@pytest.mark.parametrize("G", [4, 8])
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 8])
+def test_parity_sweep_page512(d, G, W):
+    w = small_workload(d, G, 512, W, seed=1000 + d + 10 * G + W)
+    # lengths on both sides of page boundaries: len % 512 in {0, 1, 511} and a short one
+    run_parity(w, [1024, 1537, 1023, max(W, 37)], W)
+
+
+@pytest.mark.parametrize("d", [128, 512])
+@pytest.mark.parametrize("W", [1, 5])
+def test_parity_page64(d, W):
+    w = small_workload(d, 4, 64, W, seed=2000 + d + W)
+    run_parity(w, [64 * 7, 64 * 3 + 1, 63 + W, 1000], W)
+
+
+@pytest.mark.parametrize("W", [16, 100, 512])
+def test_parity_prompt_chunks(W):
+    w = small_workload(128, 4, 512, W, seed=3000 + W)
+    run_parity(w, [W, W + 700, 1536], W)
+
+
+def test_paged_equals_identity_table_bytes():
+    w = small_workload(128, 4, 512, 4, seed=4000)
+    lens = [2000, 513, 4096]
+    case = synth.make_case(w, lens=lens)
+    a = DeviceCase(case).attend()
+    table, n_pages = synth.identity_table(case.lens, w.page_size)
+    b = DeviceCase(case, table=table, n_pages=n_pages).attend()
+    assert torch.equal(a, b)
+    # a second shuffle of the same pool contents
+    w2 = synth.Workload("sweep", 0, 2, 4, 128, 512, 4, seed=4001)
+    t2, n2, _ = synth.page_table(w2, case.lens)
+    c = DeviceCase(case, table=t2, n_pages=n2).attend()
+    assert torch.equal(a, c)
+
+
+def test_repeat_runs_are_bitwise_equal():
+    w = small_workload(512, 8, 512, 4, seed=4100, sigma=0.5)
+    case = synth.make_case(w, lens=[3000, 700, 9000])
+    dc = DeviceCase(case)
+    a = dc.attend()
+    b = dc.attend()
+    assert torch.equal(a, b)
+
+
+def test_nan_never_reaches_output_and_negative_control_goes_red():
+    w = small_workload(128, 4, 512, 2, seed=4200)
+    lens = [1300, 600]
+    case, dc, out = run_parity(w, lens, 2)
+    # spare pages and unused slots are NaN (the pool was NaN-filled); output finite.
+    spare = int(dc.table[0, -1].item()) if dc.table.shape[1] > 3 else None
+    assert torch.isfinite(out).all()
+    # negative control: point stream 0's first page at a NaN spare page -> must go red
+    t = case.table.copy()
+    _, _, spares = synth.page_table(w, case.lens)
+    t[0, 0] = spares[0]
+    bad = DeviceCase(case)
+    bad.table.copy_(torch.from_numpy(t).cuda())
+    out_bad = bad.attend()
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, 2, w.group, w.scale)
+    assert not (torch.isfinite(out_bad).all() and max_abs(out_bad, ref) <= TOL)
+
+
+def test_put_rows_bit_exact_against_host_scatter():
+    rng = np.random.default_rng(5)
+    import verify_paged_gqa_b200 as tf
+    for d, P, W in [(128, 512, 1), (128, 64, 8), (512, 512, 3), (512, 64, 5)]:
+        w = synth.Workload("put", 3, 2, 4, d, P, W, seed=6000 + d + P + W)
+        lens = np.array([W, P + 3, 3 * P], dtype=np.int32)
+        table, n_pages, _ = synth.page_table(w, lens)
+        host_k = rng.integers(0, 0x7F7F, size=(n_pages, 2, P, d)).astype(np.uint16)
+        host_v = rng.integers(0, 0x7F7F, size=(n_pages, 2, P, d)).astype(np.uint16)
+        kp, vp = bf16_tensor(host_k), bf16_tensor(host_v)
+        kr = rng.integers(0, 0xFFFF, size=(3, W, 2, d)).astype(np.uint16)
+        vr = rng.integers(0, 0xFFFF, size=(3, W, 2, d)).astype(np.uint16)
+        tf.tf_kv_put_rows(kp, vp, torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda(),
+                          bf16_tensor(kr), bf16_tensor(vr), max_len=int(lens.max()))
+        oracle.put_rows(host_k, host_v, table, lens, kr, vr)
+        got_k = kp.view(torch.int16).cpu().numpy().view(np.uint16)
+        got_v = vp.view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(got_k, host_k)
+        assert np.array_equal(got_v, host_v)
+
+
+def test_status_flags_bad_len_and_bad_page():
+    import verify_paged_gqa_b200 as tf
+    w = small_workload(128, 4, 512, 1, seed=7000)
+    case = synth.make_case(w, lens=[1000, 1500])
+    dc = DeviceCase(case)
+    ws = dc.workspace(1)
+    tf.tf_workspace_status(ws)  # clear
+    lens = torch.tensor([1000, 1500], dtype=torch.int32, device="cuda")
+    out = dc.attend(lens=lens, max_len=1200, ws=ws)   # stream 1 longer than max_len
+    flags = tf.tf_workspace_status(ws)
+    assert flags & tf.TF_DEV_BAD_LEN
+    assert torch.isnan(out[1]).all()
+    ref = oracle.attend(case.q[:1], case.k_lin[:1], case.v_lin[:1], case.lens[:1], 1, 4, w.scale)
+    assert max_abs(out[:1], ref) <= TOL
+    # a page id outside the pool is never read and is reported
+    dc.table[0, 1] = dc.k_pool.shape[0] + 5
+    dc.attend(ws=ws)
+    assert tf.tf_workspace_status(ws) & tf.TF_DEV_BAD_PAGE
+    assert tf.tf_workspace_status(ws) == 0
+
+
+def test_workspace_too_small_is_refused():
+    import verify_paged_gqa_b200 as tf
+    w = small_workload(128, 4, 512, 1, seed=7100)
+    case = synth.make_case(w, lens=[40000, 30000])
+    dc = DeviceCase(case)
+    need = dc.workspace(1).numel()
+    with pytest.raises(tf.TFError) as e:
+        dc.attend(ws=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == tf.TF_ENOSPACE

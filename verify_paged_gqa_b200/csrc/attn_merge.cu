@@ -1,0 +1,118 @@
+// attn_merge.cu -- combines the split-context partials of each row block.
+//
+// TensorFold #1620, the comment on per-tile lookup and the reply on the
+// merge: decode is split across the context by a partial kernel and put back
+// together by a merge kernel that reads no pages.  For a row with partials
+// (O_c, m_c, l_c), c = 0..nc-1 (O_c unnormalised, m_c the running max in log2
+// units, l_c the running sum relative to m_c):
+//     m* = max_c m_c,   w_c = 2^(m_c - m*),
+//     out = (sum_c w_c O_c) / (sum_c w_c l_c)
+// The maximum and the sum of l are warp-shuffle reductions; the O sum runs
+// in chunk order, so the result is the same on every run.
+//
+// One block per (stream, KV head, row block); one warp per row.  Streams
+// whose length is out of range get NaN rows (and the status bit).
+#include "launch.cuh"
+#include "plan.cuh"
+
+namespace tfp {
+
+template <int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__ AttnParams p)
+{
+    constexpr int DL = D / 32;
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int nwarps = blockDim.x / 32;
+    const int blk = blockIdx.x;
+    const int b = blk % p.n_rblk;
+    const int u = blk / p.n_rblk;
+    const int kh = u % p.Hkv;
+    const int s = u / p.Hkv;
+    const int len = __ldg(p.lens + s);
+    const int m0 = b * p.RB;
+    const int m1 = min(p.M, m0 + p.RB);
+    const float NEG_INF = -__int_as_float(0x7f800000);
+
+    if (!len_ok(p, len)) {
+        if (threadIdx.x == 0 && kh == 0 && b == 0)
+            set_flag(p.flags, kDevBadLen);
+        const float nan = __int_as_float(0x7fc00000);
+        for (int m = m0 + warp; m < m1; m += nwarps) {
+            const int wr = m / p.G;
+            const int h = kh * p.G + (m - wr * p.G);
+            float *orow = p.out + (((size_t)s * p.W + wr) * p.Hq + h) * D;
+            for (int e = lane * 4; e < D; e += 128)
+                *reinterpret_cast<float4 *>(orow + e) = make_float4(nan, nan, nan, nan);
+        }
+        return;
+    }
+    const int nc = block_chunks(p, len, b);
+    if (nc <= 1)
+        return;  // the partial kernel wrote the output itself
+    const size_t slot_floats = (size_t)p.RB * (D + 2);
+    const float *base = p.part + part_slot(p, s, kh, b, 0) * slot_floats;
+
+    for (int m = m0 + warp; m < m1; m += nwarps) {
+        const int r = m - m0;
+        float mx = NEG_INF;
+        for (int c = lane; c < nc; c += 32)
+            mx = fmaxf(mx, base[c * slot_floats + (size_t)p.RB * D + r]);
+#pragma unroll
+        for (int k = 16; k >= 1; k >>= 1)
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, k));
+        float l = 0.f;
+        for (int c = lane; c < nc; c += 32) {
+            const float mc = base[c * slot_floats + (size_t)p.RB * D + r];
+            const float lc = base[c * slot_floats + (size_t)p.RB * D + p.RB + r];
+            l += (mc == NEG_INF) ? 0.f : lc * fast_exp2(mc - mx);
+        }
+#pragma unroll
+        for (int k = 16; k >= 1; k >>= 1)
+            l += __shfl_xor_sync(0xffffffffu, l, k);
+
+        float acc[DL];
+#pragma unroll
+        for (int e = 0; e < DL; ++e)
+            acc[e] = 0.f;
+        for (int c = 0; c < nc; ++c) {
+            const float *sl = base + c * slot_floats;
+            const float mc = sl[(size_t)p.RB * D + r];
+            const float w = (mc == NEG_INF) ? 0.f : fast_exp2(mc - mx);
+            const float *orow = sl + (size_t)r * D;
+#pragma unroll
+            for (int q = 0; q < DL / 4; ++q) {
+                const float4 v = *reinterpret_cast<const float4 *>(orow + q * 128 + lane * 4);
+                acc[q * 4 + 0] = fmaf(w, v.x, acc[q * 4 + 0]);
+                acc[q * 4 + 1] = fmaf(w, v.y, acc[q * 4 + 1]);
+                acc[q * 4 + 2] = fmaf(w, v.z, acc[q * 4 + 2]);
+                acc[q * 4 + 3] = fmaf(w, v.w, acc[q * 4 + 3]);
+            }
+        }
+        const float inv = 1.f / l;
+        const int wr = m / p.G;
+        const int h = kh * p.G + (m - wr * p.G);
+        float *orow = p.out + (((size_t)s * p.W + wr) * p.Hq + h) * D;
+#pragma unroll
+        for (int q = 0; q < DL / 4; ++q)
+            *reinterpret_cast<float4 *>(orow + q * 128 + lane * 4) =
+                make_float4(acc[q * 4 + 0] * inv, acc[q * 4 + 1] * inv, acc[q * 4 + 2] * inv,
+                            acc[q * 4 + 3] * inv);
+    }
+}
+
+template <int D>
+cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream)
+{
+    const int64_t blocks = (int64_t)p.S * p.Hkv * p.n_rblk;
+    if (blocks == 0)
+        return cudaSuccess;
+    const int threads = 32 * min(8, p.RB);
+    attn_merge_kernel<D><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_attn_merge<128>(const AttnParams &, cudaStream_t);
+template cudaError_t launch_attn_merge<512>(const AttnParams &, cudaStream_t);
+
+}  // namespace tfp

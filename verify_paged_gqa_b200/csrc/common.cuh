@@ -1,0 +1,153 @@
+// common.cuh -- shared definitions for the paged-attention kernels (sm_100a).
+//
+// Inline-PTX wrappers for the pieces of the Blackwell memory pipeline the
+// kernels use: mbarriers with transaction counts, and bulk (TMA engine)
+// copies from global to shared memory that complete on an mbarrier.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace tfp {
+
+// Device-side status bits (mirrors the public TF_DEV_* values).
+constexpr uint32_t kDevBadLen = 1u;
+constexpr uint32_t kDevBadPage = 2u;
+constexpr uint32_t kDevTimeout = 4u;
+
+// The workspace starts with a 256-byte header; word 0 is the status word.
+constexpr size_t kWsHeaderBytes = 256;
+
+// Per-device bookkeeping on the host (kernel attributes set once per device).
+constexpr int kMaxDevices = 64;
+
+// A pipeline wait gives up after this many nanoseconds (an internal error:
+// every wait in these kernels is satisfied by work issued earlier in the
+// same CTA).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+struct AttnParams {
+    const __nv_bfloat16 *k_pool;
+    const __nv_bfloat16 *v_pool;
+    const int32_t *table;
+    const int32_t *lens;
+    const __nv_bfloat16 *q;
+    float *out;
+    float *part;        // split-context partials (workspace past the header)
+    uint32_t *flags;    // workspace status word
+    int32_t n_pages, Hkv, P, D;
+    int32_t table_stride, S, max_len;
+    int32_t Hq, G, W, M;        // M = G * W query rows per (stream, KV head)
+    int32_t RB, n_rblk;         // rows per row block, row blocks per unit
+    int32_t CH, max_chunks;     // keys per context chunk, chunks per row block bound
+    float scale_log2;           // scale * log2(e): scores are kept in log2 units
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete; false after the
+// time limit (the caller records kDevTimeout and winds down).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs)
+            return false;
+    }
+}
+
+// Bulk copy (TMA engine, no tensor map) of `bytes` from global to this
+// CTA's shared memory; completion is counted on `bar` in bytes.  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// L2 policy for data read once per call (K/V streams): evict first.
+__device__ __forceinline__ uint64_t l2_evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// bf16 pair (packed in a 32-bit word, low element first) to two floats.
+// bf16 is the upper half of an IEEE binary32, so widening is a shift/mask.
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ void named_barrier(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void set_flag(uint32_t *flags, uint32_t bit)
+{
+    atomicOr(flags, bit);
+}
+
+}  // namespace tfp

@@ -1,0 +1,31 @@
+// launch.cuh -- host-side launchers of the kernels (one per translation unit).
+#pragma once
+
+#include "common.cuh"
+
+namespace tfp {
+
+struct PutParams {
+    __nv_bfloat16 *k_pool;
+    __nv_bfloat16 *v_pool;
+    const int32_t *table;
+    const int32_t *lens;
+    const __nv_bfloat16 *k_rows;
+    const __nv_bfloat16 *v_rows;
+    int32_t n_pages, Hkv, P, D;
+    int32_t table_stride, S, W;
+};
+
+cudaError_t launch_kv_put(const PutParams &p, cudaStream_t stream);
+
+// Rows per row block of the CUDA-core partial kernel.
+constexpr int kSimtRows = 4;
+
+template <int D>
+size_t simt_smem_bytes();
+template <int D>
+cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream);
+template <int D>
+cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream);
+
+}  // namespace tfp

@@ -1,0 +1,283 @@
+// tf_paged.cu -- the C ABI: argument checks, the launch plan, dispatch.
+//
+// Every entry point checks its host arguments before enqueueing anything
+// and returns a TF_* status.  The plan (row blocks, context chunk, grid)
+// depends only on host arguments and the device's SM count, so a captured
+// graph stays valid while lens grow up to max_len.
+#include "../../include/tf_paged.h"
+#include "launch.cuh"
+#include "plan.cuh"
+
+#include <cmath>
+
+namespace tfp {
+namespace {
+
+int device_sm_count(int *sms)
+{
+    static int cached[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return TF_ECUDA;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            n <= 0)
+            return TF_ECUDA;
+        cached[dev] = n;
+    }
+    *sms = cached[dev];
+    return TF_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_pool_streams(const tf_kv_pool *pool, const tf_streams *st)
+{
+    if (!pool || !st)
+        return TF_EINVAL;
+    if (pool->n_pages < 1 || pool->n_kv_heads < 1 || pool->page_size < 1)
+        return TF_EINVAL;
+    if (pool->head_dim != 128 && pool->head_dim != 512)
+        return TF_EUNSUPPORTED;
+    if (pool->page_size % 64 != 0)
+        return TF_EUNSUPPORTED;
+    if (st->n_streams < 0 || st->table_stride < 1 || st->max_len < 1)
+        return TF_EINVAL;
+    if ((int64_t)st->max_len > (int64_t)st->table_stride * pool->page_size)
+        return TF_EINVAL;
+    if ((int64_t)st->n_streams * st->table_stride > INT32_MAX)
+        return TF_EINVAL;
+    if (st->n_streams > 0 && (!st->table || !st->lens))
+        return TF_EINVAL;
+    if (!pool->k_pool || !pool->v_pool || !aligned16(pool->k_pool) || !aligned16(pool->v_pool))
+        return TF_EINVAL;
+    return TF_OK;
+}
+
+struct Plan {
+    AttnParams p;
+    int grid;
+    size_t ws_bytes;
+};
+
+// Chunk length in pages: the one that minimises the busiest CTA's pages
+// (items are dealt round-robin to one CTA per SM) plus the partials' write
+// and read traffic, assuming every stream at max_len.
+int choose_chunk_pages(int64_t units, int pages_max, int grid, double partial_pages_per_item)
+{
+    int best = 1;
+    double best_cost = 1e300;
+    const int cap = pages_max < 64 ? pages_max : 64;
+    for (int cp = 1; cp <= cap; ++cp) {
+        const int64_t per_unit = (pages_max + cp - 1) / cp;
+        const int64_t items = units * per_unit;
+        const int64_t rounds = (items + grid - 1) / grid;
+        double cost = (double)rounds * cp;
+        if (per_unit > 1)
+            cost += (double)items * partial_pages_per_item / grid;
+        cost += 0.02 * (double)rounds;  // per-item fixed cost (pipeline turn, combine)
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = cp;
+        }
+    }
+    return best;
+}
+
+int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t rows,
+              int32_t rows_max, Plan *plan)
+{
+    int rc = check_pool_streams(pool, st);
+    if (rc != TF_OK)
+        return rc;
+    if (Hq < 1 || Hq % pool->n_kv_heads != 0)
+        return TF_EINVAL;
+    if (rows < 1 || rows > rows_max || st->max_len < rows)
+        return TF_EINVAL;
+    const int G = Hq / pool->n_kv_heads;
+    const int64_t M = (int64_t)G * rows;
+    if (M > (1 << 20))
+        return TF_EINVAL;
+    int sms = 0;
+    rc = device_sm_count(&sms);
+    if (rc != TF_OK)
+        return rc;
+
+    AttnParams &p = plan->p;
+    p = AttnParams{};
+    p.n_pages = pool->n_pages;
+    p.Hkv = pool->n_kv_heads;
+    p.P = pool->page_size;
+    p.D = pool->head_dim;
+    p.table_stride = st->table_stride;
+    p.S = st->n_streams;
+    p.max_len = st->max_len;
+    p.Hq = Hq;
+    p.G = G;
+    p.W = rows;
+    p.M = static_cast<int32_t>(M);
+    p.RB = kSimtRows;
+    p.n_rblk = static_cast<int32_t>((M + p.RB - 1) / p.RB);
+
+    const int pages_max = (st->max_len + p.P - 1) / p.P;
+    const int64_t units = (int64_t)p.S * p.Hkv * p.n_rblk;
+    const int grid_cap = sms;  // one persistent CTA per SM
+    const double partial_bytes = 2.0 * p.RB * (p.D + 2) * 4.0;
+    const double page_bytes = 2.0 * p.P * p.D * 2.0;
+    const int cp = choose_chunk_pages(units > 0 ? units : 1, pages_max, grid_cap,
+                                      partial_bytes / page_bytes);
+    p.CH = cp * p.P;
+    p.max_chunks = (st->max_len + p.CH - 1) / p.CH;
+    const int64_t items_max = units * p.max_chunks;
+    plan->grid = static_cast<int>(items_max < grid_cap ? (items_max > 0 ? items_max : 1) : grid_cap);
+    plan->ws_bytes = kWsHeaderBytes;
+    if (p.max_chunks > 1)
+        plan->ws_bytes += (size_t)units * p.max_chunks * p.RB * (p.D + 2) * sizeof(float);
+    return TF_OK;
+}
+
+int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32_t Hq,
+              int32_t rows, int32_t rows_max, float scale, float *out, void *ws,
+              size_t ws_bytes, void *stream)
+{
+    Plan plan;
+    int rc = make_plan(pool, st, Hq, rows, rows_max, &plan);
+    if (rc != TF_OK)
+        return rc;
+    if (!q || !out || !ws || !aligned16(q) || !aligned16(out) || !aligned16(ws))
+        return TF_EINVAL;
+    if (!std::isfinite(scale))
+        return TF_EINVAL;
+    if (ws_bytes < plan.ws_bytes)
+        return TF_ENOSPACE;
+    if (st->n_streams == 0)
+        return TF_OK;
+    AttnParams &p = plan.p;
+    p.k_pool = static_cast<const __nv_bfloat16 *>(pool->k_pool);
+    p.v_pool = static_cast<const __nv_bfloat16 *>(pool->v_pool);
+    p.table = st->table;
+    p.lens = st->lens;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.out = out;
+    p.flags = static_cast<uint32_t *>(ws);
+    p.part = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeaderBytes);
+    p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (p.D == 128) {
+        e = launch_attn_simt<128>(p, plan.grid, s);
+        if (e == cudaSuccess)
+            e = launch_attn_merge<128>(p, s);
+    } else {
+        e = launch_attn_simt<512>(p, plan.grid, s);
+        if (e == cudaSuccess)
+            e = launch_attn_merge<512>(p, s);
+    }
+    return e == cudaSuccess ? TF_OK : TF_ECUDA;
+}
+
+}  // namespace
+}  // namespace tfp
+
+using namespace tfp;
+
+extern "C" {
+
+int tf_kv_put_rows(const tf_kv_pool *pool, const tf_streams *streams, const void *k_rows,
+                   const void *v_rows, int32_t rows, void *stream)
+{
+    int rc = check_pool_streams(pool, streams);
+    if (rc != TF_OK)
+        return rc;
+    if (rows < 1 || streams->max_len < rows)
+        return TF_EINVAL;
+    if (streams->n_streams == 0)
+        return TF_OK;
+    if (!k_rows || !v_rows || !aligned16(k_rows) || !aligned16(v_rows))
+        return TF_EINVAL;
+    PutParams p;
+    p.k_pool = static_cast<__nv_bfloat16 *>(pool->k_pool);
+    p.v_pool = static_cast<__nv_bfloat16 *>(pool->v_pool);
+    p.table = streams->table;
+    p.lens = streams->lens;
+    p.k_rows = static_cast<const __nv_bfloat16 *>(k_rows);
+    p.v_rows = static_cast<const __nv_bfloat16 *>(v_rows);
+    p.n_pages = pool->n_pages;
+    p.Hkv = pool->n_kv_heads;
+    p.P = pool->page_size;
+    p.D = pool->head_dim;
+    p.table_stride = streams->table_stride;
+    p.S = streams->n_streams;
+    p.W = rows;
+    return launch_kv_put(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_ECUDA;
+}
+
+size_t tf_paged_attn_workspace_bytes(const tf_kv_pool *pool, const tf_streams *streams,
+                                     int32_t n_q_heads, int32_t rows)
+{
+    Plan plan;
+    if (make_plan(pool, streams, n_q_heads, rows, 4096, &plan) != TF_OK)
+        return 0;
+    return plan.ws_bytes;
+}
+
+int tf_paged_attn_decode(const tf_kv_pool *pool, const tf_streams *streams, const void *q,
+                         int32_t n_q_heads, float scale, float *out, void *workspace,
+                         size_t workspace_bytes, void *stream)
+{
+    return attn_call(pool, streams, q, n_q_heads, 1, 1, scale, out, workspace, workspace_bytes,
+                     stream);
+}
+
+int tf_paged_attn_verify(const tf_kv_pool *pool, const tf_streams *streams, const void *q,
+                         int32_t n_q_heads, int32_t rows, float scale, float *out,
+                         void *workspace, size_t workspace_bytes, void *stream)
+{
+    return attn_call(pool, streams, q, n_q_heads, rows, 8, scale, out, workspace,
+                     workspace_bytes, stream);
+}
+
+int tf_paged_attn_prompt(const tf_kv_pool *pool, const tf_streams *streams, const void *q,
+                         int32_t n_q_heads, int32_t rows, float scale, float *out,
+                         void *workspace, size_t workspace_bytes, void *stream)
+{
+    return attn_call(pool, streams, q, n_q_heads, rows, 4096, scale, out, workspace,
+                     workspace_bytes, stream);
+}
+
+int tf_workspace_status(void *workspace, uint32_t *flags, void *stream)
+{
+    if (!workspace || !flags)
+        return TF_EINVAL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t host = 0;
+    if (cudaMemcpyAsync(&host, workspace, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return TF_ECUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof host, s) != cudaSuccess)
+        return TF_ECUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return TF_ECUDA;
+    *flags = host;
+    return TF_OK;
+}
+
+const char *tf_status_str(int status)
+{
+    switch (status) {
+    case TF_OK:
+        return "TF_OK";
+    case TF_EINVAL:
+        return "TF_EINVAL: invalid argument";
+    case TF_EUNSUPPORTED:
+        return "TF_EUNSUPPORTED: shape not supported by this build";
+    case TF_ENOSPACE:
+        return "TF_ENOSPACE: workspace too small";
+    case TF_ECUDA:
+        return "TF_ECUDA: CUDA launch or query failed";
+    default:
+        return "unknown status";
+    }
+}
+
+}  // extern "C"
