@@ -157,7 +157,7 @@ class Workload:
         self.out = torch.empty(self.q.shape, dtype=torch.float32, device=device)
         nbytes = tf.tf_paged_attn_workspace_bytes(self.k_pool, self.v_pool, self.table, self.lens,
                                                   w.n_q_heads, W, self.max_len)
-        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         self.attn_fn = (tf.tf_paged_attn_decode if W == 1 else
                         tf.tf_paged_attn_verify if W <= 8 else tf.tf_paged_attn_prompt)
         self.bytes_per_step = kv_bytes(self.lens_np, w.n_kv_heads, w.head_dim)

@@ -118,10 +118,13 @@ TF_API int tf_kv_put_rows(const tf_kv_pool *pool, const tf_streams *streams,
                    const void *k_rows, const void *v_rows, int32_t rows,
                    void *stream);
 
-/* Workspace bytes an attention call with these arguments needs (0 on a bad
- * argument).  The workspace holds split-context partial results and the
- * status word; it needs no initialisation and may be reused by later calls
- * on the same stream. */
+/* Workspace bytes an attention call with these arguments needs on the
+ * current device (0 on a bad argument).  The workspace holds split-context
+ * partial results and, in its first 4 bytes, the device status word, which
+ * the calls only OR bits into: zero those 4 bytes once after allocating
+ * (cudaMemset, or one tf_workspace_status call).  The rest needs no
+ * initialisation.  One workspace may serve later calls on the same stream;
+ * calls that may run concurrently need separate workspaces. */
 TF_API size_t tf_paged_attn_workspace_bytes(const tf_kv_pool *pool,
                                      const tf_streams *streams,
                                      int32_t n_q_heads, int32_t rows);

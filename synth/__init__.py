@@ -132,6 +132,8 @@ WORKLOADS = {
                              len_range=(2048, 9216)),
     "prompt_9216": Workload("prompt_9216", 1, 8, 4, 128, 512, 512, seed=5, lens=(9216,),
                             prompt_len=9216),
+    # smaller copy of the batched decode for profiler captures (still > the 126 MB L2)
+    "decode_12x8k": Workload("decode_12x8k", 12, 8, 4, 128, 512, 1, seed=6, lens=(8192,) * 12),
 }
 
 

@@ -49,7 +49,7 @@ class DeviceCase:
     def workspace(self, rows):
         n = self.tf.tf_paged_attn_workspace_bytes(self.k_pool, self.v_pool, self.table, self.lens,
                                                   self.w.n_q_heads, rows, self.max_len)
-        return torch.empty(n, dtype=torch.uint8, device="cuda")
+        return torch.zeros(n, dtype=torch.uint8, device="cuda")
 
     def attend(self, q=None, lens=None, max_len=None, ws=None, out=None, kind=None):
         q = self.q if q is None else q

@@ -23,7 +23,8 @@ def lib():
     path = build.build()
     import verify_paged_gqa_b200 as t
     assert os.path.samefile(path, t.library_path)
-    return t
+    from verify_paged_gqa_b200 import _abi
+    return _abi
 
 
 def test_header_declares_the_entry_points():
@@ -50,13 +51,13 @@ def test_library_is_built_for_sm100a(lib):
 def _pool(lib, **kw):
     base = dict(k_pool=16, v_pool=16, n_pages=8, n_kv_heads=2, page_size=512, head_dim=128)
     base.update(kw)
-    return lib._abi.tf_kv_pool(**base)
+    return lib.tf_kv_pool(**base)
 
 
 def _streams(lib, **kw):
     base = dict(table=16, table_stride=4, lens=16, n_streams=2, max_len=2048)
     base.update(kw)
-    return lib._abi.tf_streams(**base)
+    return lib.tf_streams(**base)
 
 
 @pytest.mark.parametrize("pool_kw,streams_kw,hq,rows,want", [

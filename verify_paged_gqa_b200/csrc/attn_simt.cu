@@ -6,34 +6,41 @@
 // the core pool"): decode reads keys through the page table, split across
 // the context (the partial kernel) and merged (the merge kernel, which reads
 // no pages); its later comment moves the page lookup out of the per-key loop
-// to once per tile.  Here one lookup serves a whole page.
+// to once per tile.  Here each page id is read once, one page before its
+// first tile is needed.
 //
 // Layout of one CTA (persistent, one per SM):
-//   last warp     producer: walks the CTA's work items, looks each page up
-//                 once, and streams K and V tiles of TK positions into a ring
-//                 of NSTAGE shared-memory stages with bulk copies (TMA engine,
-//                 no tensor map: a tile of a page-head is one contiguous run).
-//   other warps   consumers (8 at head dim 128): tile T of the CTA's
-//                 sequence goes to consumer warp T % (number of consumers).
-//                 A warp keeps its own online-softmax state (running max m,
-//                 running sum l, unnormalised O) for the four rows of the
-//                 item; at the end of the item the warps' states are combined
-//                 through shared memory and the item's result is written:
-//                 the normalised output when the row block has one chunk,
-//                 else a partial for the merge kernel.
+//   last warp     producer (one lane): walks the CTA's work items one item
+//                 ahead; per item it copies the four query rows into a
+//                 double-buffered shared slot and streams K and V tiles of TK
+//                 positions into a ring of NSTAGE stages with bulk copies
+//                 (TMA engine, no tensor map: a tile of one page and KV head
+//                 is one contiguous run).  Page ids are read one page early.
+//   other warps   consumers: tile T of the CTA's sequence goes to consumer
+//                 warp T % NCW.  A warp keeps its own online-softmax state
+//                 (running max m, running sum l, unnormalised O) for the four
+//                 rows of the item.  At the end of the item each warp parks
+//                 its state in shared memory; the last warp to arrive
+//                 combines them and writes the item's result (the normalised
+//                 output when the row block has one chunk, else a partial for
+//                 the merge kernel).  No CTA-wide barrier: the other warps go
+//                 straight on to the next item.
 //
 // Inner loop of a consumer warp on one tile (head dim 128, TK = 32):
 //   scores  the warp is 4 groups of 8 lanes; group g takes 8 keys, lane i of
-//           a group holds 16 of the 128 dims of the 4 query rows (fp32 in
-//           registers) and accumulates 8 keys x 4 rows partial dots; three
-//           butterfly rounds (reduce-scatter over the 8 lanes) leave lane L
-//           with the 4 rows' full scores of key L.
+//           a group holds 16 of the 128 dims of the 4 query rows as packed
+//           bf16 pairs and accumulates 8 keys x 4 rows partial dots with
+//           bf16 x bf16 -> fp32 FMAs (fma.rn.f32.bf16: exact products, fp32
+//           sums, no conversions); three butterfly rounds (reduce-scatter
+//           over the 8 lanes) leave lane L with the 4 rows' full scores of
+//           key L.
 //   softmax tile max per row by warp shuffles, exp2 of log2-scaled scores;
 //           masked positions are SELECTED to -inf (never multiplied), so NaN
 //           in unused slots cannot leak.
-//   PV      lane L owns dims 4L..4L+3 of the 4 output rows; probabilities
-//           come from a small per-warp shared buffer; only positions below
-//           the item's end are visited, so no unused slot is ever read.
+//   PV      lane L owns dims 4L..4L+3 of the 4 output rows as fp32 pairs and
+//           updates them with packed fp32 FMAs (two per instruction);
+//           probabilities come from a per-warp shared buffer; only positions
+//           below the item's end are visited, so no unused slot is read.
 // Head dim 512 uses TK = 8 and one group of 32 lanes; the same steps.
 #include "launch.cuh"
 #include "plan.cuh"
@@ -44,7 +51,6 @@ template <int D>
 struct SimtCfg;
 // Registers are split per SM sub-partition: with 9 warps one sub-partition
 // holds 3 warps (at most 168 registers each), with 8 warps 2 (255 each).
-// Head dim 512 keeps 64 output accumulators per lane and takes 7 consumers.
 template <>
 struct SimtCfg<128> {
     static constexpr int TK = 32;      // positions per tile
@@ -68,15 +74,20 @@ template <int D>
 struct SimtSmem {
     static constexpr int TK = SimtCfg<D>::TK;
     static constexpr int NSTAGE = SimtCfg<D>::NSTAGE;
+    static constexpr int NCW = SimtCfg<D>::NCW;
     static constexpr int TILE_BYTES = TK * D * 2;
     alignas(128) uint8_t kv[NSTAGE][2][TILE_BYTES];
-    static constexpr int NCW = SimtCfg<D>::NCW;
-    alignas(16) float pbuf[NCW][TK * kR];
-    alignas(16) float wo[NCW][kR][D];
+    alignas(16) __nv_bfloat16 qbuf[2][kR][D];      // the item's query rows (double buffer)
+    alignas(16) float pbuf[NCW][TK][2 * kR];        // per key: p0,p0,p1,p1,p2,p2,p3,p3
+    alignas(16) float wo[NCW][kR][D];               // parked warp states
     float wm[NCW][kR];
     float wl[NCW][kR];
     uint64_t full[NSTAGE];
     uint64_t empty[NSTAGE];
+    uint64_t q_full[2];
+    uint64_t q_empty[2];
+    uint64_t w_free;       // the parked-state slot is free again (combine done)
+    int w_count;           // warps parked for the current item
     volatile int abort_flag;
 };
 
@@ -102,54 +113,126 @@ __device__ __forceinline__ float warp_sum(float v, int lo_mask)
     return v;
 }
 
+// c + a.lo * b.lo + a.hi * b.hi for two packed bf16 pairs; each step is one
+// fp32 FMA of an exact bf16 x bf16 product.
+__device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c)
+{
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\t"
+        "mov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "+f"(c)
+        : "r"(a), "r"(b));
+    return c;
+}
+
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) { return make_float2(bf_lo(w), bf_hi(w)); }
+
+// A bounded wait that turns a timeout into the abort state of the CTA.
+template <int D>
+__device__ __forceinline__ bool wait_or_abort(SimtSmem<D> &sm, uint64_t *bar, uint32_t parity,
+                                              uint32_t *flags)
+{
+    if (sm.abort_flag)
+        return false;
+    if (mbar_wait(bar, parity))
+        return true;
+    set_flag(flags, kDevTimeout);
+    sm.abort_flag = 1;
+    return false;
+}
+
+// Copies the four query rows of item `it` into q slot (j & 1).
+template <int D>
+__device__ __forceinline__ bool producer_q(const AttnParams &p, SimtSmem<D> &sm,
+                                           const WorkItem &it, uint32_t j, uint64_t pol)
+{
+    const int slot = j & 1;
+    if (!wait_or_abort(sm, &sm.q_empty[slot], ((j >> 1) & 1u) ^ 1u, p.flags))
+        return false;
+    mbar_arrive_expect_tx(&sm.q_full[slot], kR * D * 2);
+    for (int r = 0; r < kR; ++r) {
+        const int mm = min(it.b * kR + r, p.M - 1);
+        const int wr = mm / p.G;
+        const int h = it.kh * p.G + (mm - wr * p.G);
+        bulk_g2s(sm.qbuf[slot][r], p.q + (((size_t)it.s * p.W + wr) * p.Hq + h) * D, D * 2,
+                 &sm.q_full[slot], pol);
+    }
+    return true;
+}
+
+// One lane.  Looks one item ahead: the next item's query rows are copied
+// when the current item starts, and every page id is read one page before
+// its first tile, so no table read sits on the copy path.
 template <int D>
 __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &sm)
 {
     constexpr int TK = SimtCfg<D>::TK;
     constexpr int NSTAGE = SimtCfg<D>::NSTAGE;
     const uint64_t pol = l2_evict_first_policy();
-    ItemCursor cur;
+    ItemCursor cur, ahead;
     cur.init();
-    WorkItem it;
+    ahead.init();
+    WorkItem it, nx;
     uint32_t T = 0;
-    bool aborted = false;
-    for (int64_t i = blockIdx.x; !aborted && cur.seek(p, i, it); i += gridDim.x) {
+    uint32_t j = 0;  // item counter of this CTA
+    int64_t i = blockIdx.x;
+    uint32_t q_issued = 0;  // items whose query copy was started
+    bool have = cur.seek(p, i, it);
+    if (have && producer_q<D>(p, sm, it, 0, pol))
+        q_issued = 1;
+    int32_t page_next = have ? __ldg(p.table + (int64_t)it.s * p.table_stride + it.key0 / p.P) : 0;
+    while (have && !sm.abort_flag) {
+        const bool have_nx = ahead.seek(p, i + gridDim.x, nx);
+        if (have_nx && producer_q<D>(p, sm, nx, j + 1, pol))
+            q_issued = j + 2;
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
-        int lp_cached = -1;
-        int32_t page = 0;
-        for (int t0 = it.key0; t0 < it.key1; t0 += TK, ++T) {
-            const int stage = T % NSTAGE;
-            const uint32_t ph = (T / NSTAGE) & 1u;
-            if (!mbar_wait(&sm.empty[stage], ph ^ 1u)) {
-                set_flag(p.flags, kDevTimeout);
-                sm.abort_flag = 1;
-                aborted = true;
-                break;
-            }
-            const int lp = t0 / p.P;
-            if (lp != lp_cached) {  // one table read per page
-                page = __ldg(trow + lp);
-                lp_cached = lp;
-            }
-            const int nk = min(TK, it.key1 - t0);
-            const uint32_t bytes = static_cast<uint32_t>(nk) * D * 2u;
-            if (page >= 0 && page < p.n_pages) {
-                const size_t off = (((size_t)page * p.Hkv + it.kh) * p.P + (t0 - lp * p.P)) * D;
-                mbar_arrive_expect_tx(&sm.full[stage], 2u * bytes);
-                bulk_g2s(sm.kv[stage][0], p.k_pool + off, bytes, &sm.full[stage], pol);
-                bulk_g2s(sm.kv[stage][1], p.v_pool + off, bytes, &sm.full[stage], pol);
-            } else {
+        const int lp_end = (it.key1 + p.P - 1) / p.P;
+        for (int lp = it.key0 / p.P; lp < lp_end && !sm.abort_flag; ++lp) {
+            const int32_t page = page_next;
+            if (lp + 1 < lp_end)
+                page_next = __ldg(trow + lp + 1);
+            else if (have_nx)
+                page_next = __ldg(p.table + (int64_t)nx.s * p.table_stride + nx.key0 / p.P);
+            const bool page_ok = page >= 0 && page < p.n_pages;
+            if (!page_ok)
                 set_flag(p.flags, kDevBadPage);
-                mbar_arrive(&sm.full[stage]);
+            const int pos0 = max(it.key0, lp * p.P);
+            const int pos1 = min(it.key1, (lp + 1) * p.P);
+            const size_t base = (((size_t)(page_ok ? page : 0) * p.Hkv + it.kh) * p.P) * D;
+            for (int t0 = pos0; t0 < pos1; t0 += TK, ++T) {
+                const int stage = T % NSTAGE;
+                if (!wait_or_abort(sm, &sm.empty[stage], ((T / NSTAGE) & 1u) ^ 1u, p.flags))
+                    break;
+                const int nk = min(TK, pos1 - t0);
+                const uint32_t bytes = static_cast<uint32_t>(nk) * D * 2u;
+                if (page_ok) {
+                    const size_t off = base + (size_t)(t0 - lp * p.P) * D;
+                    mbar_arrive_expect_tx(&sm.full[stage], 2u * bytes);
+                    bulk_g2s(sm.kv[stage][0], p.k_pool + off, bytes, &sm.full[stage], pol);
+                    bulk_g2s(sm.kv[stage][1], p.v_pool + off, bytes, &sm.full[stage], pol);
+                } else {
+                    mbar_arrive(&sm.full[stage]);
+                }
             }
         }
+        have = have_nx;
+        it = nx;
+        cur = ahead;
+        i += gridDim.x;
+        ++j;
     }
-    if (aborted) {
+    if (sm.abort_flag) {
         // Let every copy this CTA started land before the CTA can exit.
         const uint32_t n = T < (uint32_t)NSTAGE ? T : (uint32_t)NSTAGE;
         for (uint32_t k = 1; k <= n; ++k) {
             const uint32_t t = T - k;
             (void)mbar_wait(&sm.full[t % NSTAGE], (t / NSTAGE) & 1u);
+        }
+        for (uint32_t k = 1; k <= 2 && k <= q_issued; ++k) {
+            const uint32_t jj = q_issued - k;  // the last two query copies started
+            (void)mbar_wait(&sm.q_full[jj & 1], (jj >> 1) & 1u);
         }
     }
 }
@@ -161,13 +244,15 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
     constexpr int TK = SimtCfg<D>::TK;
     constexpr int NSTAGE = SimtCfg<D>::NSTAGE;
     constexpr int LG = SimtCfg<D>::LG;
+    constexpr int NCW = SimtCfg<D>::NCW;
     constexpr int NG = 32 / LG;        // key groups per warp
     constexpr int KPG = TK / NG;       // keys per group
     constexpr int NACC = KPG * kR;     // partial dots per lane
     constexpr int NV = NACC / LG;      // full scores per lane after the reduce-scatter
     constexpr int CPL = D / 8 / LG;    // 16-byte chunks of a key row per lane
     constexpr int DL = D / 32;         // output dims per lane
-    constexpr int kNCW = SimtCfg<D>::NCW;
+    constexpr int LOG_LG = (LG == 8) ? 3 : 5;
+    static_assert((1 << LOG_LG) == LG, "lane group");
     static_assert(NACC == 32 && CPL == 2, "tile shape");
     static_assert(NV == kR || NV == 1, "score ownership");
 
@@ -179,58 +264,56 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
     cur.init();
     WorkItem it;
     uint32_t T0 = 0;  // CTA tile index of the item's first tile
+    uint32_t j = 0;
 
-    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x) {
-        // --- this item's query rows, fp32 in registers --------------------
-        float qv[kR][CPL * 8];
+    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
+        // --- this item's query rows: packed bf16 pairs in registers --------
+        uint32_t qh[kR][CPL * 4];
         int lim[kR];
+        {
+            const int slot = j & 1;
+            const bool ok = wait_or_abort(sm, &sm.q_full[slot], (j >> 1) & 1u, p.flags);
 #pragma unroll
-        for (int r = 0; r < kR; ++r) {
-            const int m = it.b * kR + r;
-            const int mm = min(m, p.M - 1);
-            const int wr = mm / p.G;
-            const int h = it.kh * p.G + (mm - wr * p.G);
-            lim[r] = row_lim(p, it.len, m);
-            const __nv_bfloat16 *qrow = p.q + (((size_t)it.s * p.W + wr) * p.Hq + h) * D;
+            for (int r = 0; r < kR; ++r) {
+                const int m = it.b * kR + r;
+                lim[r] = row_lim(p, it.len, m);
+                const bool live = ok && m < p.M;
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(qrow + (li + c * LG) * 8);
-                const bool live = m < p.M;
-                qv[r][c * 8 + 0] = live ? bf_lo(w.x) : 0.f;
-                qv[r][c * 8 + 1] = live ? bf_hi(w.x) : 0.f;
-                qv[r][c * 8 + 2] = live ? bf_lo(w.y) : 0.f;
-                qv[r][c * 8 + 3] = live ? bf_hi(w.y) : 0.f;
-                qv[r][c * 8 + 4] = live ? bf_lo(w.z) : 0.f;
-                qv[r][c * 8 + 5] = live ? bf_hi(w.z) : 0.f;
-                qv[r][c * 8 + 6] = live ? bf_lo(w.w) : 0.f;
-                qv[r][c * 8 + 7] = live ? bf_hi(w.w) : 0.f;
+                for (int c = 0; c < CPL; ++c) {
+                    const uint4 w =
+                        *reinterpret_cast<const uint4 *>(&sm.qbuf[slot][r][(li + c * LG) * 8]);
+                    qh[r][c * 4 + 0] = live ? w.x : 0u;
+                    qh[r][c * 4 + 1] = live ? w.y : 0u;
+                    qh[r][c * 4 + 2] = live ? w.z : 0u;
+                    qh[r][c * 4 + 3] = live ? w.w : 0u;
+                }
             }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.q_empty[slot]);
         }
 
-        float m_run[kR], l_lane[NV], o[kR][DL];
+        float m_run[kR], l_lane[NV];
+        float2 o2[kR][DL / 2];
 #pragma unroll
         for (int r = 0; r < kR; ++r) {
             m_run[r] = NEG_INF;
 #pragma unroll
-            for (int e = 0; e < DL; ++e)
-                o[r][e] = 0.f;
+            for (int e = 0; e < DL / 2; ++e)
+                o2[r][e] = make_float2(0.f, 0.f);
         }
 #pragma unroll
-        for (int j = 0; j < NV; ++j)
-            l_lane[j] = 0.f;
+        for (int jj = 0; jj < NV; ++jj)
+            l_lane[jj] = 0.f;
 
         const int ntiles = (it.key1 - it.key0 + TK - 1) / TK;
-        int t = (warp - (int)(T0 % kNCW) + kNCW) % kNCW;
-        for (; t < ntiles; t += kNCW) {
+        int t = (warp - (int)(T0 % NCW) + NCW) % NCW;
+        for (; t < ntiles; t += NCW) {
             const uint32_t T = T0 + t;
             const int stage = T % NSTAGE;
-            if (!sm.abort_flag && !mbar_wait(&sm.full[stage], (T / NSTAGE) & 1u)) {
-                if (lane == 0)
-                    set_flag(p.flags, kDevTimeout);
-                sm.abort_flag = 1;
-            }
+            const bool ok = wait_or_abort(sm, &sm.full[stage], (T / NSTAGE) & 1u, p.flags);
             __syncwarp();
-            if (sm.abort_flag)
+            if (!ok)
                 continue;
             const uint8_t *Ks = sm.kv[stage][0];
             const uint8_t *Vs = sm.kv[stage][1];
@@ -249,14 +332,13 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 for (int kk = 0; kk < KPG; ++kk) {
                     const uint4 w = *reinterpret_cast<const uint4 *>(
                         Ks + (grp * KPG + kk) * D * 2 + chunk * 16);
-                    const float kf[8] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y),
-                                         bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w)};
 #pragma unroll
                     for (int r = 0; r < kR; ++r) {
                         float a = acc[kk * kR + r];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            a = fmaf(qv[r][c * 8 + e], kf[e], a);
+                        a = fma_bf16x2(qh[r][c * 4 + 0], w.x, a);
+                        a = fma_bf16x2(qh[r][c * 4 + 1], w.y, a);
+                        a = fma_bf16x2(qh[r][c * 4 + 2], w.z, a);
+                        a = fma_bf16x2(qh[r][c * 4 + 3], w.w, a);
                         acc[kk * kR + r] = a;
                     }
                 }
@@ -265,8 +347,6 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
             // Round with mask msk keeps the upper half of the array in lanes
             // whose bit msk is set.  Afterwards lane li holds entries
             // x = li * NV + j (j < NV) of the original kk * kR + r numbering.
-            constexpr int LOG_LG = (LG == 8) ? 3 : 5;
-            static_assert((1 << LOG_LG) == LG, "lane group");
 #pragma unroll
             for (int rnd = 0; rnd < LOG_LG; ++rnd) {
                 const int msk = LG >> (rnd + 1);
@@ -312,7 +392,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 alpha[r] = fast_exp2(m_run[r] - m_use[r]);
                 m_run[r] = mn;
             }
-            float *pb = sm.pbuf[warp];
+            float *pb = &sm.pbuf[warp][0][0];
             if constexpr (NV == kR) {
                 float pr[kR];
 #pragma unroll
@@ -320,48 +400,53 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                     pr[r] = fast_exp2(sc[r] - m_use[r]);
                     l_lane[r] = fmaf(l_lane[r], alpha[r], pr[r]);
                 }
-                *reinterpret_cast<float4 *>(pb + lane * 4) = make_float4(pr[0], pr[1], pr[2], pr[3]);
+                float4 *dst = reinterpret_cast<float4 *>(pb + lane * 2 * kR);
+                dst[0] = make_float4(pr[0], pr[0], pr[1], pr[1]);
+                dst[1] = make_float4(pr[2], pr[2], pr[3], pr[3]);
             } else {
                 const int r = li & 3;
                 const float mu = r == 0 ? m_use[0] : r == 1 ? m_use[1] : r == 2 ? m_use[2] : m_use[3];
                 const float al = r == 0 ? alpha[0] : r == 1 ? alpha[1] : r == 2 ? alpha[2] : alpha[3];
                 const float pr = fast_exp2(sc[0] - mu);
                 l_lane[0] = fmaf(l_lane[0], al, pr);
-                pb[lane] = pr;
+                *reinterpret_cast<float2 *>(pb + lane * 2) = make_float2(pr, pr);
             }
             __syncwarp();
 
             // --- O = alpha * O + P V over the visited positions -----------
 #pragma unroll
-            for (int r = 0; r < kR; ++r)
+            for (int r = 0; r < kR; ++r) {
+                const float2 a2 = make_float2(alpha[r], alpha[r]);
 #pragma unroll
-                for (int e = 0; e < DL; ++e)
-                    o[r][e] *= alpha[r];
+                for (int e = 0; e < DL / 2; ++e)
+                    o2[r][e] = __fmul2_rn(o2[r][e], a2);
+            }
 
             auto pv_step = [&](int kk) {
-                const float4 pr = *reinterpret_cast<const float4 *>(pb + kk * 4);
-                const float prr[4] = {pr.x, pr.y, pr.z, pr.w};
+                const float4 pa = *reinterpret_cast<const float4 *>(pb + kk * 2 * kR);
+                const float4 pc = *reinterpret_cast<const float4 *>(pb + kk * 2 * kR + 4);
+                const float2 pr[4] = {make_float2(pa.x, pa.y), make_float2(pa.z, pa.w),
+                                      make_float2(pc.x, pc.y), make_float2(pc.z, pc.w)};
                 if constexpr (D == 128) {
                     const uint2 w = *reinterpret_cast<const uint2 *>(Vs + kk * D * 2 + lane * 8);
-                    const float v[4] = {bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y)};
+                    const float2 v01 = bf2_to_f2(w.x), v23 = bf2_to_f2(w.y);
 #pragma unroll
-                    for (int r = 0; r < kR; ++r)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o[r][e] = fmaf(prr[r], v[e], o[r][e]);
+                    for (int r = 0; r < kR; ++r) {
+                        o2[r][0] = __ffma2_rn(pr[r], v01, o2[r][0]);
+                        o2[r][1] = __ffma2_rn(pr[r], v23, o2[r][1]);
+                    }
                 } else {
                     const uint4 w0 = *reinterpret_cast<const uint4 *>(Vs + kk * D * 2 + lane * 16);
                     const uint4 w1 =
                         *reinterpret_cast<const uint4 *>(Vs + kk * D * 2 + D + lane * 16);
-                    const float v[16] = {bf_lo(w0.x), bf_hi(w0.x), bf_lo(w0.y), bf_hi(w0.y),
-                                         bf_lo(w0.z), bf_hi(w0.z), bf_lo(w0.w), bf_hi(w0.w),
-                                         bf_lo(w1.x), bf_hi(w1.x), bf_lo(w1.y), bf_hi(w1.y),
-                                         bf_lo(w1.z), bf_hi(w1.z), bf_lo(w1.w), bf_hi(w1.w)};
+                    const float2 v[8] = {bf2_to_f2(w0.x), bf2_to_f2(w0.y), bf2_to_f2(w0.z),
+                                         bf2_to_f2(w0.w), bf2_to_f2(w1.x), bf2_to_f2(w1.y),
+                                         bf2_to_f2(w1.z), bf2_to_f2(w1.w)};
 #pragma unroll
                     for (int r = 0; r < kR; ++r)
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            o[r][e] = fmaf(prr[r], v[e], o[r][e]);
+                        for (int e = 0; e < 8; ++e)
+                            o2[r][e] = __ffma2_rn(pr[r], v[e], o2[r][e]);
                 }
             };
             if (nk == TK) {
@@ -379,7 +464,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
         }
         T0 += ntiles;
 
-        // --- combine the eight warp states of this item ---------------------
+        // --- park this warp's state; the last warp in combines -------------
         float l_row[kR];
         if constexpr (NV == kR) {
 #pragma unroll
@@ -391,6 +476,8 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
             for (int r = 0; r < kR; ++r)
                 l_row[r] = __shfl_sync(0xffffffffu, lr, r);
         }
+        // the slot is free once the previous item's combine is done
+        (void)wait_or_abort(sm, &sm.w_free, (j & 1u) ^ 1u, p.flags);
         if (lane == 0) {
 #pragma unroll
             for (int r = 0; r < kR; ++r) {
@@ -402,59 +489,86 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
         for (int r = 0; r < kR; ++r) {
             if constexpr (D == 128) {
                 *reinterpret_cast<float4 *>(&sm.wo[warp][r][lane * 4]) =
-                    make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
+                    make_float4(o2[r][0].x, o2[r][0].y, o2[r][1].x, o2[r][1].y);
             } else {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     *reinterpret_cast<float4 *>(&sm.wo[warp][r][h * 256 + lane * 8]) =
-                        make_float4(o[r][h * 8 + 0], o[r][h * 8 + 1], o[r][h * 8 + 2],
-                                    o[r][h * 8 + 3]);
+                        make_float4(o2[r][h * 4 + 0].x, o2[r][h * 4 + 0].y, o2[r][h * 4 + 1].x,
+                                    o2[r][h * 4 + 1].y);
                     *reinterpret_cast<float4 *>(&sm.wo[warp][r][h * 256 + lane * 8 + 4]) =
-                        make_float4(o[r][h * 8 + 4], o[r][h * 8 + 5], o[r][h * 8 + 6],
-                                    o[r][h * 8 + 7]);
+                        make_float4(o2[r][h * 4 + 2].x, o2[r][h * 4 + 2].y, o2[r][h * 4 + 3].x,
+                                    o2[r][h * 4 + 3].y);
                 }
             }
         }
-        named_barrier(1, kNCW * 32);
-        // Element pairs of the kR x D block, dealt over the consumer threads.
-        for (int e2 = warp * 32 + lane; e2 < kR * D / 2; e2 += kNCW * 32) {
-            const int e0 = 2 * e2;
-            const int r = e0 / D;
-            const int col = e0 - r * D;
+        __syncwarp();
+        int arrived = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            arrived = atomicAdd(&sm.w_count, 1);
+        }
+        arrived = __shfl_sync(0xffffffffu, arrived, 0);
+        if (arrived != NCW - 1)
+            continue;
+
+        // --- this warp is the last one in: combine the NCW states ----------
+        if (lane == 0)
+            sm.w_count = 0;
+        __threadfence_block();
+#pragma unroll 1
+        for (int r = 0; r < kR; ++r) {
             const int m = it.b * kR + r;
             float mstar = NEG_INF;
 #pragma unroll
-            for (int w = 0; w < kNCW; ++w)
+            for (int w = 0; w < NCW; ++w)
                 mstar = fmaxf(mstar, sm.wm[w][r]);
-            float lstar = 0.f, v0 = 0.f, v1 = 0.f;
+            float wt[NCW];
+            float lstar = 0.f;
 #pragma unroll
-            for (int w = 0; w < kNCW; ++w) {
+            for (int w = 0; w < NCW; ++w) {
                 const float mw = sm.wm[w][r];
-                const float wt = (mw == NEG_INF) ? 0.f : fast_exp2(mw - mstar);
-                lstar = fmaf(sm.wl[w][r], wt, lstar);
-                const float2 ov = *reinterpret_cast<const float2 *>(&sm.wo[w][r][col]);
-                v0 = fmaf(ov.x, wt, v0);
-                v1 = fmaf(ov.y, wt, v1);
+                wt[w] = (mw == NEG_INF) ? 0.f : fast_exp2(mw - mstar);
+                lstar = fmaf(sm.wl[w][r], wt[w], lstar);
             }
-            if (m < p.M && !sm.abort_flag) {
-                if (it.nc == 1) {
-                    const int wr = m / p.G;
-                    const int h = it.kh * p.G + (m - wr * p.G);
-                    float *orow = p.out + (((size_t)it.s * p.W + wr) * p.Hq + h) * D;
-                    const float inv = 1.f / lstar;
-                    *reinterpret_cast<float2 *>(orow + col) = make_float2(v0 * inv, v1 * inv);
-                } else {
-                    float *slot = p.part + part_slot(p, it.s, it.kh, it.b, it.c) *
-                                               (size_t)(p.RB * (D + 2));
-                    *reinterpret_cast<float2 *>(slot + (size_t)r * D + col) = make_float2(v0, v1);
-                    if (col == 0) {
-                        slot[(size_t)p.RB * D + r] = mstar;
-                        slot[(size_t)p.RB * D + p.RB + r] = lstar;
-                    }
+            if (m >= p.M || sm.abort_flag)
+                continue;
+            float *dst;
+            float scale_out;
+            if (it.nc == 1) {
+                const int wr = m / p.G;
+                const int h = it.kh * p.G + (m - wr * p.G);
+                dst = p.out + (((size_t)it.s * p.W + wr) * p.Hq + h) * D;
+                scale_out = 1.f / lstar;
+            } else {
+                float *slot =
+                    p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(p.RB * (D + 2));
+                dst = slot + (size_t)r * D;
+                scale_out = 1.f;
+                if (lane == 0) {
+                    slot[(size_t)p.RB * D + r] = mstar;
+                    slot[(size_t)p.RB * D + p.RB + r] = lstar;
                 }
             }
+#pragma unroll
+            for (int q4 = 0; q4 < D / 128; ++q4) {
+                const int col = q4 * 128 + lane * 4;
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int w = 0; w < NCW; ++w) {
+                    const float4 v = *reinterpret_cast<const float4 *>(&sm.wo[w][r][col]);
+                    a.x = fmaf(v.x, wt[w], a.x);
+                    a.y = fmaf(v.y, wt[w], a.y);
+                    a.z = fmaf(v.z, wt[w], a.z);
+                    a.w = fmaf(v.w, wt[w], a.w);
+                }
+                *reinterpret_cast<float4 *>(dst + col) =
+                    make_float4(a.x * scale_out, a.y * scale_out, a.z * scale_out, a.w * scale_out);
+            }
         }
-        named_barrier(1, kNCW * 32);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&sm.w_free);
     }
 }
 
@@ -471,6 +585,12 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.q_full[s], 1);
+            mbar_init(&sm.q_empty[s], SimtCfg<D>::NCW);
+        }
+        mbar_init(&sm.w_free, 1);
+        sm.w_count = 0;
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -478,9 +598,8 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
     if (warp == SimtCfg<D>::NCW) {
         if (lane == 0)
             simt_producer<D>(p, sm);
-        return;
-    }
-    simt_consumer<D>(p, sm, warp, lane);
+    } else
+        simt_consumer<D>(p, sm, warp, lane);
 }
 
 // Host-side launcher (same translation unit as the kernel template).
