@@ -178,9 +178,12 @@ class Workload:
         self.attend()
 
     def check_flags(self):
+        torch = self.torch
+        site = int(self.ws[4:8].view(torch.int32).item())   # which wait gave up, if any
+        self.ws[4:8].zero_()
         flags = self.tf.tf_workspace_status(self.ws)
         if flags:
-            raise RuntimeError(f"device status word set: {flags:#x}")
+            raise RuntimeError(f"device status word set: {flags:#x} (wait sites {site:#x})")
 
 
 def time_steps(wl, steps, warmup, barrier, sampler=None):

@@ -84,6 +84,13 @@ struct SimtSmem {
     float wl[NCW][kR];
     uint64_t full[NSTAGE];
     uint64_t empty[NSTAGE];
+    // Tile each stage was last armed for.  Consumers take tiles round-robin
+    // and the ring is deeper than the number of consumers, so a warp can
+    // reach stage s for tile T while the stage's previous tile (T - NSTAGE,
+    // another warp's) is still in flight; a parity wait alone cannot tell
+    // those phases apart.  The tag can: it moves to T only after tile
+    // T - NSTAGE has been consumed.
+    volatile uint32_t stage_tile[NSTAGE];
     uint64_t q_full[2];
     uint64_t q_empty[2];
     uint64_t w_free;       // the parked-state slot is free again (combine done)
@@ -132,15 +139,38 @@ __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) { return make_float2(bf_
 // A bounded wait that turns a timeout into the abort state of the CTA.
 template <int D>
 __device__ __forceinline__ bool wait_or_abort(SimtSmem<D> &sm, uint64_t *bar, uint32_t parity,
-                                              uint32_t *flags)
+                                              uint32_t *flags, uint32_t site)
 {
     if (sm.abort_flag)
         return false;
     if (mbar_wait(bar, parity))
         return true;
     set_flag(flags, kDevTimeout);
+    set_flag(flags + 1, site);
     sm.abort_flag = 1;
     return false;
+}
+
+// Waits until stage `stage` has been armed for tile T (bounded like the
+// mbarrier waits); after that its full barrier's parity refers to tile T.
+template <int D>
+__device__ __forceinline__ bool wait_tag(SimtSmem<D> &sm, int stage, uint32_t T, uint32_t *flags)
+{
+    if (sm.stage_tile[stage] == T)
+        return true;
+    const long long t0 = clock64();
+    while (sm.stage_tile[stage] != T) {
+        if (sm.abort_flag)
+            return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            set_flag(flags, kDevTimeout);
+            set_flag(flags + 1, kWaitTag);
+            sm.abort_flag = 1;
+            return false;
+        }
+        __nanosleep(32);
+    }
+    return true;
 }
 
 // Copies the four query rows of item `it` into q slot (j & 1).
@@ -149,7 +179,7 @@ __device__ __forceinline__ bool producer_q(const AttnParams &p, SimtSmem<D> &sm,
                                            const WorkItem &it, uint32_t j, uint64_t pol)
 {
     const int slot = j & 1;
-    if (!wait_or_abort(sm, &sm.q_empty[slot], ((j >> 1) & 1u) ^ 1u, p.flags))
+    if (!wait_or_abort(sm, &sm.q_empty[slot], ((j >> 1) & 1u) ^ 1u, p.flags, kWaitQEmpty))
         return false;
     mbar_arrive_expect_tx(&sm.q_full[slot], kR * D * 2);
     for (int r = 0; r < kR; ++r) {
@@ -203,8 +233,9 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
             const size_t base = (((size_t)(page_ok ? page : 0) * p.Hkv + it.kh) * p.P) * D;
             for (int t0 = pos0; t0 < pos1; t0 += TK, ++T) {
                 const int stage = T % NSTAGE;
-                if (!wait_or_abort(sm, &sm.empty[stage], ((T / NSTAGE) & 1u) ^ 1u, p.flags))
+                if (!wait_or_abort(sm, &sm.empty[stage], ((T / NSTAGE) & 1u) ^ 1u, p.flags, kWaitEmpty))
                     break;
+                sm.stage_tile[stage] = T;
                 const int nk = min(TK, pos1 - t0);
                 const uint32_t bytes = static_cast<uint32_t>(nk) * D * 2u;
                 if (page_ok) {
@@ -272,7 +303,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
         int lim[kR];
         {
             const int slot = j & 1;
-            const bool ok = wait_or_abort(sm, &sm.q_full[slot], (j >> 1) & 1u, p.flags);
+            const bool ok = wait_or_abort(sm, &sm.q_full[slot], (j >> 1) & 1u, p.flags, kWaitQFull);
 #pragma unroll
             for (int r = 0; r < kR; ++r) {
                 const int m = it.b * kR + r;
@@ -311,7 +342,8 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
         for (; t < ntiles; t += NCW) {
             const uint32_t T = T0 + t;
             const int stage = T % NSTAGE;
-            const bool ok = wait_or_abort(sm, &sm.full[stage], (T / NSTAGE) & 1u, p.flags);
+            const bool ok = wait_tag<D>(sm, stage, T, p.flags) &&
+                            wait_or_abort(sm, &sm.full[stage], (T / NSTAGE) & 1u, p.flags, kWaitFull);
             __syncwarp();
             if (!ok)
                 continue;
@@ -477,7 +509,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 l_row[r] = __shfl_sync(0xffffffffu, lr, r);
         }
         // the slot is free once the previous item's combine is done
-        (void)wait_or_abort(sm, &sm.w_free, (j & 1u) ^ 1u, p.flags);
+        (void)wait_or_abort(sm, &sm.w_free, (j & 1u) ^ 1u, p.flags, kWaitFree);
         if (lane == 0) {
 #pragma unroll
             for (int r = 0; r < kR; ++r) {
@@ -584,6 +616,7 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
         for (int s = 0; s < SimtSmem<D>::NSTAGE; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+            sm.stage_tile[s] = 0xffffffffu;
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.q_full[s], 1);

@@ -22,10 +22,18 @@ constexpr size_t kWsHeaderBytes = 256;
 // Per-device bookkeeping on the host (kernel attributes set once per device).
 constexpr int kMaxDevices = 64;
 
-// A pipeline wait gives up after this many nanoseconds (an internal error:
-// every wait in these kernels is satisfied by work issued earlier in the
-// same CTA).
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// A pipeline wait gives up after this many SM clock cycles (about two
+// seconds at B200 clocks; an internal error: every wait in these kernels is
+// satisfied by work issued earlier in the same CTA).  The SM's own cycle
+// counter is used because it only moves forward.
+constexpr long long kWaitLimitCycles = 4000000000ll;
+
+// Word 1 of the workspace header records which wait gave up (one bit per
+// site), for diagnosis; word 0 is the status word.
+enum WaitSite : uint32_t {
+    kWaitFull = 1u, kWaitEmpty = 2u, kWaitQFull = 4u, kWaitQEmpty = 8u, kWaitFree = 16u,
+    kWaitTag = 32u
+};
 
 struct AttnParams {
     const __nv_bfloat16 *k_pool;
@@ -47,13 +55,6 @@ struct AttnParams {
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t global_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
@@ -98,11 +99,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity))
         return true;
-    const uint64_t t0 = global_ns();
+    const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs)
+        if ((it & 255u) == 0 && clock64() - t0 > kWaitLimitCycles)
             return false;
     }
 }

@@ -281,3 +281,4 @@ const char *tf_status_str(int status)
 }
 
 }  // extern "C"
+
