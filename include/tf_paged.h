@@ -152,6 +152,29 @@ TF_API int tf_paged_attn_prompt(const tf_kv_pool *pool, const tf_streams *stream
                          float scale, float *out, void *workspace,
                          size_t workspace_bytes, void *stream);
 
+/* Single-row decode that allocates nothing and takes no workspace.  The
+ * source pages have no counterpart of this call.
+ * For callers that cannot allocate device memory for a workspace: a
+ * plug-in hosted by an engine that hands it only its input and output
+ * buffers, or a serving loop that must not call cudaMalloc once running.
+ * The split-context scratch is one static device array of 8 MiB inside
+ * this library, held by every GPU that loads it until the process exits.
+ * Arguments, results and errors are those of tf_paged_attn_decode, except:
+ *  - TF_ENOSPACE when the call would need more than the 8 MiB of scratch
+ *    (tf_paged_attn_workspace_bytes with rows = 1 gives the need);
+ *  - the first call on each device looks the array's device address up
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device;
+ *  - every call on a device shares the one array, which keeps the last
+ *    call's contents: calls whose kernels may overlap on the GPU (other
+ *    streams, other host threads) race and must be serialised by the caller;
+ *  - device-side status bits are not reported (streams with a bad length
+ *    still get NaN outputs); use tf_paged_attn_decode to read them. */
+TF_API int tf_paged_attn_decode_noalloc(const tf_kv_pool *pool,
+                                        const tf_streams *streams,
+                                        const void *q, int32_t n_q_heads,
+                                        float scale, float *out, void *stream);
+
 /* Reads the workspace's device status word (TF_DEV_* bits accumulated by
  * the attention calls since the last read) into *flags and clears it.
  * Synchronises `stream`.  Returns TF_OK, TF_EINVAL or TF_ECUDA. */

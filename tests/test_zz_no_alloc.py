@@ -1,0 +1,71 @@
+"""tf_paged_attn_decode_noalloc: the decode entry point that allocates nothing.
+
+Callers that cannot allocate device memory (a plug-in that only receives its
+input and output buffers from the engine hosting it, or a serving loop that
+must not call cudaMalloc once running) use this call; its split-context
+scratch is a static array inside the library.  This file runs last, so a
+failure here leaves every other test already run.  It checks, through the C
+ABI, that two calls in a row give the workspace entry point's output.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_cases import TOL, DeviceCase
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(tf, dc, q, out):
+    from verify_paged_gqa_b200 import _abi
+    fn = tf.raw.tf_paged_attn_decode_noalloc
+    fn.argtypes = [ctypes.POINTER(_abi.tf_kv_pool), ctypes.POINTER(_abi.tf_streams),
+                   ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_void_p,
+                   ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    pool = _abi.tf_kv_pool(dc.k_pool.data_ptr(), dc.v_pool.data_ptr(), *dc.k_pool.shape)
+    st = _abi.tf_streams(dc.table.data_ptr(), dc.table.shape[1], dc.lens.data_ptr(),
+                         dc.table.shape[0], dc.max_len)
+    return fn(ctypes.byref(pool), ctypes.byref(st), q.data_ptr(), q.shape[2],
+              float(dc.w.scale), out.data_ptr(),
+              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("d,G,lens", [(128, 4, [40960, 9000, 513]), (512, 8, [3000, 9216])])
+def test_noalloc_decode_matches_workspace_decode_twice(d, G, lens):
+    import verify_paged_gqa_b200 as tf
+    w = synth.Workload("noalloc", 0, 2, G, d, 512, 1, seed=8000 + d)
+    case = synth.make_case(w, lens=lens)
+    dc = DeviceCase(case)
+    ref = dc.attend(kind="decode")
+    for _ in range(2):
+        out = torch.full(dc.q.shape, float("nan"), dtype=torch.float32, device="cuda")
+        assert _noalloc(tf, dc, dc.q, out) == tf.TF_OK
+        torch.cuda.synchronize()
+        assert torch.isfinite(out).all()
+        assert float((out - ref).abs().max()) <= TOL
+
+
+def test_noalloc_refuses_a_plan_beyond_its_scratch():
+    import verify_paged_gqa_b200 as tf
+    # 64 streams x 8 KV heads at 131,072 positions needs far more than 8 MiB of partials
+    w = synth.Workload("noalloc_big", 0, 8, 4, 128, 512, 1, seed=8100)
+    S, L = 64, 131072
+    pages = S * (L // 512)
+    k_pool = torch.empty((1, 8, 512, 128), dtype=torch.bfloat16, device="cuda")
+    table = torch.zeros((S, L // 512), dtype=torch.int32, device="cuda")
+    lens = torch.full((S,), L, dtype=torch.int32, device="cuda")
+    q = torch.zeros((S, 1, 32, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+
+    class _DC:
+        pass
+    dc = _DC()
+    dc.k_pool = dc.v_pool = k_pool
+    dc.table, dc.lens, dc.max_len, dc.w = table, lens, L, w
+    need = tf.tf_paged_attn_workspace_bytes(k_pool, k_pool, table, lens, 32, 1, L)
+    assert need > (8 << 20) and pages > 0
+    assert _noalloc(tf, dc, q, out) == tf.TF_ENOSPACE

@@ -9,6 +9,7 @@
 #include "plan.cuh"
 
 #include <cmath>
+#include <mutex>
 
 namespace tfp {
 namespace {
@@ -282,3 +283,72 @@ const char *tf_status_str(int status)
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------
+// Decode without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory for a workspace: a plug-in
+// hosted by an inference engine that hands it only its input and output
+// buffers and owns every allocation itself, or a serving loop that must not
+// call cudaMalloc once it is running (cudaMalloc can synchronise the device
+// and can fail under memory pressure).  For them the split-context scratch
+// lives in one file-scope device array of kStaticScratchBytes, which every
+// GPU that loads this library keeps until the process exits.
+namespace tfp {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB per device
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+// Device address of g_decode_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so its device address is
+// looked up once per device (with that device current) and cached.
+int static_scratch_address(void **out)
+{
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return TF_ECUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
+            return TF_ECUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return TF_OK;
+}
+
+}  // namespace
+}  // namespace tfp
+
+extern "C" int tf_paged_attn_decode_noalloc(const tf_kv_pool *pool, const tf_streams *streams,
+                                            const void *q, int32_t n_q_heads, float scale,
+                                            float *out, void *stream)
+{
+    using namespace tfp;
+    Plan plan;
+    int rc = make_plan(pool, streams, n_q_heads, 1, 1, &plan);
+    if (rc != TF_OK)
+        return rc;
+    if (!q || !out || !aligned16(q) || !aligned16(out) || !std::isfinite(scale))
+        return TF_EINVAL;
+    if (plan.ws_bytes > kStaticScratchBytes)
+        return TF_ENOSPACE;
+    void *ws = nullptr;
+    rc = static_scratch_address(&ws);
+    if (rc != TF_OK)
+        return rc;
+    if (streams->n_streams == 0)
+        return TF_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // The status word is the only part of the scratch that must start at
+    // zero (the kernels OR bits into it); the partials are written before
+    // they are read.
+    if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess)
+        return TF_ECUDA;
+    return attn_call(pool, streams, q, n_q_heads, 1, 1, scale, out, ws, kStaticScratchBytes,
+                     stream);
+}
