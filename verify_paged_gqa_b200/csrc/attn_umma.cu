@@ -1,0 +1,629 @@
+// attn_umma.cu -- split-context paged attention on the 5th-generation tensor
+// cores (tcgen05 / TMEM) for row blocks of up to 128 query rows: draft-verify
+// windows and chunked prompt rows, head dim 128.
+//
+// TensorFold #1620 ("Kolibri-1's full layers take their K/V from pages of
+// the core pool"), opening comment, "Reads": prompt rows and drafted verify
+// rows attend over keys read through the page table; TensorFold #2730 ("an
+// eight-row verify window"), "What this changes": a window holds up to eight
+// rows.  With G query heads per KV head and W window rows, the G * W rows of
+// one (stream, KV head) form a dense tile that shares every K and V row, so
+// QK^T and PV run as tensor-core MMAs here.
+//
+// One persistent CTA per SM, six warps:
+//   warp 0     producer (one lane): for each 64-position tile, one page id
+//              (read one page early) and four TMA loads (K and V, two
+//              64-dim halves each, 128-byte swizzle) into a 4-stage ring.
+//   warp 1     MMA issuer (one lane): S = Q K^T (M 128, N 64, K 128) into
+//              one of two TMEM S buffers; O += P_hi V + P_lo V (M 128, N 128,
+//              K 64) into the TMEM O accumulator.  Also owns the TMEM
+//              allocation, and zeroes V rows past the stream's end before PV
+//              (so no NaN from unused slots reaches the MMA: 0 * NaN = NaN).
+//   warps 2-5  softmax (one query row per thread, the row's TMEM lane): write
+//              the row's query into the swizzled Q tile at the start of each
+//              item; per tile, read the S row from TMEM, select masked
+//              positions to -inf, update the running max m and sum l in log2
+//              units, and write P as two bf16 parts (P = hi + lo, so the PV
+//              product keeps ~16 bits of each probability, as the fp32 CUDA
+//              core path does).  O in TMEM is rescaled only when the row max
+//              grows by more than 2^8 (exact: the final O / l does not depend
+//              on the reference max).  At the end of the item the row is
+//              normalised and stored, or left as a partial for the merge.
+#include "launch.cuh"
+#include "plan.cuh"
+
+#include <cuda.h>
+
+namespace tfp {
+
+namespace {
+
+constexpr int UD = 128;        // head dim of this kernel
+constexpr int UM = 128;        // MMA rows (the row block, padded)
+constexpr int UN = 64;         // positions per tile
+constexpr int NST = 4;         // K/V ring stages
+constexpr int kUmmaThreads = 192;
+constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more
+
+// Shared memory (SW128 regions are 1024-byte aligned).
+struct UmmaSmem {
+    // per stage: K half 0, K half 1, V half 0, V half 1; each [64 pos][64 dims] bf16
+    alignas(1024) uint8_t kv[NST][4][UN * 128];
+    alignas(1024) uint8_t q[2][UM * 128];           // two 64-dim atoms of [128 rows][64]
+    alignas(1024) uint8_t p[2][UM * 128];           // P_hi, P_lo: [128 rows][64 pos]
+    uint64_t kv_full[NST];
+    uint64_t kv_empty[NST];
+    uint64_t q_full;       // softmax warps wrote the item's Q tile
+    uint64_t q_free;       // the item's last QK MMA is done with Q
+    uint64_t s_full[2];
+    uint64_t s_free[2];
+    uint64_t p_full;       // softmax warps wrote P for the tile
+    uint64_t o_done;       // PV of the tile finished (P buffer free, O readable)
+    uint64_t fin;          // every MMA this CTA issued has completed
+    uint32_t tmem_base;
+    volatile uint32_t stage_tile[NST];
+    volatile int abort_flag;
+};
+
+constexpr size_t kUmmaSmemBytes = sizeof(UmmaSmem) + 1024;  // + alignment slack
+
+struct UmmaArgs {
+    AttnParams p;
+    CUtensorMap kmap;
+    CUtensorMap vmap;
+};
+
+__device__ __forceinline__ bool uwait(UmmaSmem &sm, uint64_t *bar, uint32_t parity, uint32_t *flags,
+                                      uint32_t site)
+{
+    if (sm.abort_flag)
+        return false;
+    if (mbar_wait(bar, parity))
+        return true;
+    set_flag(flags, kDevTimeout);
+    set_flag(flags + 1, site);
+    sm.abort_flag = 1;
+    return false;
+}
+
+__device__ __forceinline__ bool utag(UmmaSmem &sm, int stage, uint32_t T, uint32_t *flags)
+{
+    const long long t0 = clock64();
+    while (sm.stage_tile[stage] != T) {
+        if (sm.abort_flag)
+            return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            set_flag(flags, kDevTimeout);
+            set_flag(flags + 1, kWaitTag);
+            sm.abort_flag = 1;
+            return false;
+        }
+        __nanosleep(32);
+    }
+    return true;
+}
+
+// ---- tcgen05 / TMA wrappers ------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2),
+// Blackwell version field 1.  Offsets in bytes.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor for kind::f16: bf16 A and B, fp32 D.
+__host__ __device__ constexpr uint32_t f16_idesc(int M, int N, int a_mn_major, int b_mn_major)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) |
+           ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 32 bits, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Byte offset of 16-byte chunk c of row r in a [rows][64 bf16] SW128 region.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c)
+{
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---- roles -------------------------------------------------------------------
+
+__device__ __forceinline__ void umma_producer(const UmmaArgs &a, UmmaSmem &sm)
+{
+    const AttnParams &p = a.p;
+    const uint64_t pol = l2_evict_first_policy();
+    ItemCursor cur, ahead;
+    cur.init();
+    ahead.init();
+    WorkItem it, nx;
+    uint32_t T = 0;
+    int64_t i = blockIdx.x;
+    bool have = cur.seek(p, i, it);
+    int32_t page_next = have ? __ldg(p.table + (int64_t)it.s * p.table_stride + it.key0 / p.P) : 0;
+    while (have && !sm.abort_flag) {
+        const bool have_nx = ahead.seek(p, i + gridDim.x, nx);
+        const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
+        const int lp_end = (it.key1 + p.P - 1) / p.P;
+        for (int lp = it.key0 / p.P; lp < lp_end && !sm.abort_flag; ++lp) {
+            const int32_t page = page_next;
+            if (lp + 1 < lp_end)
+                page_next = __ldg(trow + lp + 1);
+            else if (have_nx)
+                page_next = __ldg(p.table + (int64_t)nx.s * p.table_stride + nx.key0 / p.P);
+            const bool page_ok = page >= 0 && page < p.n_pages;
+            if (!page_ok)
+                set_flag(p.flags, kDevBadPage);
+            const int pos0 = max(it.key0, lp * p.P);
+            const int pos1 = min(it.key1, (lp + 1) * p.P);
+            const int row0 = ((page_ok ? page : 0) * p.Hkv + it.kh) * p.P - lp * p.P;
+            for (int t0 = pos0; t0 < pos1; t0 += UN, ++T) {
+                const int st = T % NST;
+                if (!uwait(sm, &sm.kv_empty[st], ((T / NST) & 1u) ^ 1u, p.flags, kWaitEmpty))
+                    break;
+                sm.stage_tile[st] = T;
+                if (page_ok) {
+                    mbar_arrive_expect_tx(&sm.kv_full[st], 4u * UN * 128u);
+                    const int y = row0 + t0;
+                    tma_load_2d(sm.kv[st][0], &a.kmap, 0, y, &sm.kv_full[st], pol);
+                    tma_load_2d(sm.kv[st][1], &a.kmap, 64, y, &sm.kv_full[st], pol);
+                    tma_load_2d(sm.kv[st][2], &a.vmap, 0, y, &sm.kv_full[st], pol);
+                    tma_load_2d(sm.kv[st][3], &a.vmap, 64, y, &sm.kv_full[st], pol);
+                } else {
+                    mbar_arrive(&sm.kv_full[st]);
+                }
+            }
+        }
+        have = have_nx;
+        it = nx;
+        i += gridDim.x;
+    }
+    if (sm.abort_flag) {
+        const uint32_t n = T < (uint32_t)NST ? T : (uint32_t)NST;
+        for (uint32_t k = 1; k <= n; ++k) {
+            const uint32_t t = T - k;
+            (void)mbar_wait(&sm.kv_full[t % NST], (t / NST) & 1u);
+        }
+    }
+}
+
+// The whole MMA warp runs this (lane 0 issues; all lanes zero V tails).
+__device__ __forceinline__ void umma_issuer(const UmmaArgs &a, UmmaSmem &sm, int lane)
+{
+    const AttnParams &p = a.p;
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t tS[2] = {tmem, tmem + UN};
+    const uint32_t tO = tmem + 2 * UN;
+    constexpr uint32_t idQK = f16_idesc(UM, UN, 0, 0);
+    constexpr uint32_t idPV = f16_idesc(UM, UD, 0, 1);
+    const uint32_t qa = smem_addr(sm.q[0]);
+    const uint32_t pa[2] = {smem_addr(sm.p[0]), smem_addr(sm.p[1])};
+
+    ItemCursor cur;
+    cur.init();
+    WorkItem it;
+    uint32_t T0 = 0, j = 0, tt = 0;  // tt: tiles seen by this CTA (S buffer / P phases)
+    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
+        const int ntiles = (it.key1 - it.key0 + UN - 1) / UN;
+        bool ok = uwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
+        tc_fence_after();
+        // S(t) for t = 0, then per t: S(t+1), then O += P(t) V(t)
+        auto issue_qk = [&](int t) -> bool {
+            const uint32_t T = T0 + t;
+            const int st = T % NST;
+            const uint32_t u = tt + t;  // CTA-wide tile count
+            bool good = utag(sm, st, T, p.flags) && uwait(sm, &sm.kv_full[st], (T / NST) & 1u, p.flags, kWaitFull);
+            good = good && uwait(sm, &sm.s_free[u & 1], ((u >> 1) & 1u) ^ 1u, p.flags, kWaitFree);
+            tc_fence_after();
+            // positions past the stream's end: zero those V rows (both halves)
+            const int tpos = it.key0 + t * UN;
+            const int nvalid = min(UN, it.len - tpos);
+            if (good && nvalid < UN) {
+                for (int r = nvalid + (lane >> 3); r < UN; r += 4) {
+                    const int c = lane & 7;
+                    *reinterpret_cast<uint4 *>(sm.kv[st][2] + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(sm.kv[st][3] + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
+                }
+                fence_async_smem();
+            }
+            __syncwarp();
+            if (good && lane == 0) {
+                const uint32_t ka = smem_addr(sm.kv[st][0]);
+#pragma unroll
+                for (int s = 0; s < UD / 16; ++s) {
+                    const uint32_t off = (uint32_t)((s >> 2) * (UM * 128) + (s & 3) * 32);
+                    const uint32_t koff = (uint32_t)((s >> 2) * (UN * 128) + (s & 3) * 32);
+                    umma_f16(tS[u & 1], sw128_desc(qa + off, 16, 1024), sw128_desc(ka + koff, 16, 1024),
+                             idQK, s > 0);
+                }
+                umma_commit(&sm.s_full[u & 1]);
+                if (t == ntiles - 1)
+                    umma_commit(&sm.q_free);
+            }
+            __syncwarp();
+            return good;
+        };
+        if (ok)
+            ok = issue_qk(0);
+        for (int t = 0; t < ntiles; ++t) {
+            const uint32_t T = T0 + t;
+            const int st = T % NST;
+            const uint32_t u = tt + t;
+            if (ok && t + 1 < ntiles)
+                ok = issue_qk(t + 1);
+            ok = ok && uwait(sm, &sm.p_full, u & 1u, p.flags, kWaitQEmpty);
+            tc_fence_after();
+            if (ok && lane == 0) {
+                const uint32_t va = smem_addr(sm.kv[st][2]);
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                    for (int s = 0; s < UN / 16; ++s) {
+                        umma_f16(tO, sw128_desc(pa[part] + s * 32, 16, 1024),
+                                 sw128_desc(va + s * 2048, UN * 128, 1024), idPV,
+                                 (t > 0 || part > 0 || s > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit(&sm.o_done);
+                umma_commit(&sm.kv_empty[st]);
+            }
+            __syncwarp();
+        }
+        T0 += ntiles;
+        tt += ntiles;
+    }
+    // every MMA issued by this thread has completed once `fin` flips
+    if (lane == 0) {
+        umma_commit(&sm.fin);
+        (void)mbar_wait(&sm.fin, 0);
+    }
+    __syncwarp();
+}
+
+__device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, int warp, int lane)
+{
+    const AttnParams &p = a.p;
+    const int row = (warp & 3) * 32 + lane;           // TMEM lane == MMA row
+    const uint32_t lane_base = sm.tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t tS[2] = {lane_base, lane_base + UN};
+    const uint32_t tO = lane_base + 2 * UN;
+    const float NEG_INF = -__int_as_float(0x7f800000);
+
+    ItemCursor cur;
+    cur.init();
+    WorkItem it;
+    uint32_t j = 0, tt = 0;
+    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
+        const int m = it.b * UM + row;
+        const bool live = m < p.M;
+        const int lim = row_lim(p, it.len, m);
+        // --- the row's query into the swizzled Q tile ----------------------
+        bool ok = uwait(sm, &sm.q_free, (j & 1u) ^ 1u, p.flags, kWaitQEmpty);
+        {
+            const int mm = min(m, p.M - 1);
+            const int wr = mm / p.G;
+            const int h = it.kh * p.G + (mm - wr * p.G);
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.q + (((size_t)it.s * p.W + wr) * p.Hq + h) * UD);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 v = live ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(sm.q[c >> 3] + sw128_off(row, c & 7)) = v;
+            }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&sm.q_full);
+
+        float m_run = NEG_INF, l_run = 0.f;
+        const int ntiles = (it.key1 - it.key0 + UN - 1) / UN;
+        for (int t = 0; t < ntiles; ++t) {
+            const uint32_t u = tt + t;
+            const int tpos = it.key0 + t * UN;
+            ok = uwait(sm, &sm.s_full[u & 1], (u >> 1) & 1u, p.flags, kWaitFull) && ok;
+            tc_fence_after();
+            float s[UN];
+#pragma unroll
+            for (int c = 0; c < UN / 16; ++c) {
+                uint32_t r[16];
+                tmem_ld16(tS[u & 1] + c * 16, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    s[c * 16 + e] = __uint_as_float(r[e]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.s_free[u & 1]);
+            // masked, log2-scaled scores and the tile max
+            float tmax = NEG_INF;
+#pragma unroll
+            for (int e = 0; e < UN; ++e) {
+                const bool vis = live && (tpos + e) < lim && (tpos + e) < it.key1;
+                s[e] = vis ? s[e] * p.scale_log2 : NEG_INF;
+                tmax = fmaxf(tmax, s[e]);
+            }
+            // a new reference max only when the row max grows by more than 2^8
+            const bool grow = tmax > m_run + kRescaleLog2 || (m_run == NEG_INF && tmax != NEG_INF);
+            const float m_new = grow ? tmax : m_run;
+            const float m_use = m_new == NEG_INF ? 0.f : m_new;
+            const float alpha = fast_exp2(m_run - m_use);   // 0 when m_run is -inf
+            // P buffer and O: wait for the previous tile's PV
+            if (t > 0)
+                ok = uwait(sm, &sm.o_done, (u - 1) & 1u, p.flags, kWaitEmpty) && ok;
+            tc_fence_after();
+            // tcgen05.ld/st are warp-collective: rescale when any row of the
+            // warp needs it, by 1 in the rows that do not
+            const bool need = grow && t > 0 && m_run != NEG_INF;
+            if (__any_sync(0xffffffffu, need)) {
+                const float f = need ? alpha : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < UD / 16; ++c) {
+                    uint32_t r[16];
+                    tmem_ld16(tO + c * 16, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+                    tmem_st16(tO + c * 16, r);
+                }
+                tmem_wait_st();
+            }
+            if (grow)
+                l_run *= alpha;
+            m_run = m_new;
+            // P = exp2(s - m) as hi + lo bf16 parts, into the swizzled P tiles
+            float lsum = 0.f;
+#pragma unroll
+            for (int c = 0; c < UN / 8; ++c) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = fast_exp2(s[c * 8 + 2 * e] - m_use);
+                    const float p1 = fast_exp2(s[c * 8 + 2 * e + 1] - m_use);
+                    lsum += p0 + p1;
+                    hi[e] = pack_bf16(p0, p1);
+                    const float h0 = __uint_as_float(hi[e] << 16);
+                    const float h1 = __uint_as_float(hi[e] & 0xffff0000u);
+                    lo[e] = pack_bf16(p0 - h0, p1 - h1);
+                }
+                *reinterpret_cast<uint4 *>(sm.p[0] + sw128_off(row, c)) =
+                    make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(sm.p[1] + sw128_off(row, c)) =
+                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            l_run += lsum;
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.p_full);
+        }
+        // --- the item's last PV, then the row's result ----------------------
+        const uint32_t ulast = tt + ntiles - 1;
+        ok = uwait(sm, &sm.o_done, ulast & 1u, p.flags, kWaitEmpty) && ok;
+        tc_fence_after();
+        const bool write = live && ok && !sm.abort_flag;
+        float *dst = nullptr;
+        float sc = 1.f;
+        if (write) {
+            if (it.nc == 1) {
+                const int wr = m / p.G;
+                const int h = it.kh * p.G + (m - wr * p.G);
+                dst = p.out + (((size_t)it.s * p.W + wr) * p.Hq + h) * UD;
+                sc = 1.f / l_run;
+            } else {
+                float *slot = p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(p.RB * (UD + 2));
+                dst = slot + (size_t)row * UD;
+                slot[(size_t)p.RB * UD + row] = m_run;
+                slot[(size_t)p.RB * UD + p.RB + row] = l_run;
+            }
+        }
+#pragma unroll 1
+        for (int c = 0; c < UD / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(tO + c * 16, r);   // warp-collective: every lane loads
+            tmem_wait_ld();
+            if (write) {
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(dst + c * 16 + e) =
+                        make_float4(__uint_as_float(r[e]) * sc, __uint_as_float(r[e + 1]) * sc,
+                                    __uint_as_float(r[e + 2]) * sc, __uint_as_float(r[e + 3]) * sc);
+            }
+        }
+        tc_fence_before();
+        tt += ntiles;
+    }
+}
+
+__global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid_constant__ UmmaArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    UmmaSmem &sm = *reinterpret_cast<UmmaSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+            sm.stage_tile[s] = 0xffffffffu;
+        }
+        mbar_init(&sm.q_full, 4);
+        mbar_init(&sm.q_free, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.s_full[s], 1);
+            mbar_init(&sm.s_free[s], 4);
+        }
+        mbar_init(&sm.p_full, 4);
+        mbar_init(&sm.o_done, 1);
+        mbar_init(&sm.fin, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {  // TMEM: 2 S buffers (64 columns each) + O (128 columns)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                         smem_addr(&sm.tmem_base))
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == 0) {
+        if (lane == 0)
+            umma_producer(a, sm);
+        __syncwarp();
+    } else if (warp == 1) {
+        umma_issuer(a, sm, lane);
+    } else {
+        umma_softmax(a, sm, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(sm.tmem_base)
+                     : "memory");
+    }
+}
+
+// ---- host side ---------------------------------------------------------------
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                 const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn()
+{
+    static EncodeTiled fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(f);
+    }
+    return fn;
+}
+
+bool make_pool_map(CUtensorMap *map, const void *pool, const AttnParams &p)
+{
+    EncodeTiled enc = encode_fn();
+    if (!enc)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)UD, (cuuint64_t)p.n_pages * p.Hkv * p.P};
+    const cuuint64_t strides[1] = {(cuuint64_t)UD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)UN};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(pool), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int umma_rows() { return UM; }
+
+bool umma_supported(int D, int P) { return D == UD && P % UN == 0; }
+
+cudaError_t launch_attn_umma(const AttnParams &p, int grid, cudaStream_t stream)
+{
+    UmmaArgs a;
+    a.p = p;
+    if (!make_pool_map(&a.kmap, p.k_pool, p) || !make_pool_map(&a.vmap, p.v_pool, p))
+        return cudaErrorInvalidValue;
+    static bool configured[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kUmmaSmemBytes);
+        if (e != cudaSuccess)
+            return e;
+        configured[dev] = true;
+    }
+    attn_umma_kernel<<<grid, kUmmaThreads, kUmmaSmemBytes, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace tfp

@@ -60,6 +60,7 @@ struct Plan {
     AttnParams p;
     int grid;
     size_t ws_bytes;
+    bool umma;  // tensor-core partial kernel (else the CUDA-core one)
 };
 
 // Chunk length in pages: the one that minimises the busiest CTA's pages
@@ -118,7 +119,10 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     p.G = G;
     p.W = rows;
     p.M = static_cast<int32_t>(M);
-    p.RB = kSimtRows;
+    // More than one CUDA-core row block of rows sharing a KV head: a dense
+    // QK^T / PV tile for the tensor cores.
+    plan->umma = M > kSimtRows && umma_supported(p.D, p.P);
+    p.RB = plan->umma ? umma_rows() : kSimtRows;
     p.n_rblk = static_cast<int32_t>((M + p.RB - 1) / p.RB);
 
     const int pages_max = (st->max_len + p.P - 1) / p.P;
@@ -166,7 +170,11 @@ int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (p.D == 128) {
+    if (plan.umma) {
+        e = launch_attn_umma(p, plan.grid, s);
+        if (e == cudaSuccess)
+            e = launch_attn_merge<128>(p, s);
+    } else if (p.D == 128) {
         e = launch_attn_simt<128>(p, plan.grid, s);
         if (e == cudaSuccess)
             e = launch_attn_merge<128>(p, s);
