@@ -132,8 +132,10 @@ WORKLOADS = {
                              len_range=(2048, 9216)),
     "prompt_9216": Workload("prompt_9216", 1, 8, 4, 128, 512, 512, seed=5, lens=(9216,),
                             prompt_len=9216),
-    # smaller copy of the batched decode for profiler captures (still > the 126 MB L2)
+    # smaller copies of the decode and verify workloads for profiler captures
+    # (still larger than the 126 MB L2)
     "decode_12x8k": Workload("decode_12x8k", 12, 8, 4, 128, 512, 1, seed=6, lens=(8192,) * 12),
+    "verify_4x16k": Workload("verify_4x16k", 4, 4, 8, 128, 512, 8, seed=7, lens=(16384,) * 4),
 }
 
 

@@ -10,12 +10,15 @@
 // The maximum and the sum of l are warp-shuffle reductions; the O sum runs
 // in chunk order, so the result is the same on every run.
 //
-// One block per (stream, KV head, row block); one warp per row.  Streams
-// whose length is out of range get NaN rows (and the status bit).
+// One block per (stream, KV head, row block, group of up to 8 rows); one
+// warp per row.  Streams whose length is out of range get NaN rows (and the
+// status bit).
 #include "launch.cuh"
 #include "plan.cuh"
 
 namespace tfp {
+
+constexpr int kMergeRows = 8;  // rows (warps) per merge block
 
 template <int D>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__ AttnParams p)
@@ -24,18 +27,23 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int nwarps = blockDim.x / 32;
+    const int groups = (p.RB + kMergeRows - 1) / kMergeRows;
     const int blk = blockIdx.x;
-    const int b = blk % p.n_rblk;
-    const int u = blk / p.n_rblk;
+    const int g = blk % groups;
+    const int b = (blk / groups) % p.n_rblk;
+    const int u = blk / groups / p.n_rblk;
     const int kh = u % p.Hkv;
     const int s = u / p.Hkv;
     const int len = __ldg(p.lens + s);
-    const int m0 = b * p.RB;
-    const int m1 = min(p.M, m0 + p.RB);
+    const int mb = b * p.RB;                       // first row of the row block
+    const int m0 = mb + g * kMergeRows;
+    const int m1 = min(min(p.M, mb + p.RB), m0 + kMergeRows);
+    if (m0 >= m1)
+        return;
     const float NEG_INF = -__int_as_float(0x7f800000);
 
     if (!len_ok(p, len)) {
-        if (threadIdx.x == 0 && kh == 0 && b == 0)
+        if (threadIdx.x == 0 && kh == 0 && b == 0 && g == 0)
             set_flag(p.flags, kDevBadLen);
         const float nan = __int_as_float(0x7fc00000);
         for (int m = m0 + warp; m < m1; m += nwarps) {
@@ -54,7 +62,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
     const float *base = p.part + part_slot(p, s, kh, b, 0) * slot_floats;
 
     for (int m = m0 + warp; m < m1; m += nwarps) {
-        const int r = m - m0;
+        const int r = m - mb;
         float mx = NEG_INF;
         for (int c = lane; c < nc; c += 32)
             mx = fmaxf(mx, base[c * slot_floats + (size_t)p.RB * D + r]);
@@ -104,10 +112,11 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
 template <int D>
 cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream)
 {
-    const int64_t blocks = (int64_t)p.S * p.Hkv * p.n_rblk;
+    const int groups = (p.RB + kMergeRows - 1) / kMergeRows;
+    const int64_t blocks = (int64_t)p.S * p.Hkv * p.n_rblk * groups;
     if (blocks == 0)
         return cudaSuccess;
-    const int threads = 32 * min(8, p.RB);
+    const int threads = 32 * min(kMergeRows, p.RB);
     attn_merge_kernel<D><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p);
     return cudaGetLastError();
 }

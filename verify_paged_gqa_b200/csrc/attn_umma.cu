@@ -13,7 +13,7 @@
 // One persistent CTA per SM, six warps:
 //   warp 0     producer (one lane): for each 64-position tile, one page id
 //              (read one page early) and four TMA loads (K and V, two
-//              64-dim halves each, 128-byte swizzle) into a 4-stage ring.
+//              64-dim halves each, 128-byte swizzle) into a 7-stage ring.
 //   warp 1     MMA issuer (one lane): S = Q K^T (M 128, N 64, K 128) into
 //              one of two TMEM S buffers; O += P_hi V + P_lo V (M 128, N 128,
 //              K 64) into the TMEM O accumulator.  Also owns the TMEM
@@ -23,9 +23,12 @@
 //              the row's query into the swizzled Q tile at the start of each
 //              item; per tile, read the S row from TMEM, select masked
 //              positions to -inf, update the running max m and sum l in log2
-//              units, and write P as two bf16 parts (P = hi + lo, so the PV
-//              product keeps ~16 bits of each probability, as the fp32 CUDA
-//              core path does).  O in TMEM is rescaled only when the row max
+//              units, and write P into TMEM as two bf16 parts (P = hi + lo,
+//              each the truncated upper half of a float, so the PV product
+//              keeps ~15 bits of each probability, close to the fp32 CUDA
+//              core path).  Q and P live in TMEM and both MMAs
+//              read their A operand from there, so shared memory holds only
+//              the K/V ring (7 stages).  O in TMEM is rescaled only when the row max
 //              grows by more than 2^8 (exact: the final O / l does not depend
 //              on the reference max).  At the end of the item the row is
 //              normalised and stored, or left as a partial for the merge.
@@ -40,28 +43,24 @@ namespace {
 
 constexpr int UD = 128;        // head dim of this kernel
 constexpr int UM = 128;        // MMA rows (the row block, padded)
-constexpr int UN = 64;         // positions per tile
-constexpr int NST = 4;         // K/V ring stages
+constexpr int UN = 128;        // positions per tile
+constexpr int NST = 3;         // K/V ring stages (64 KB each)
 constexpr int kUmmaThreads = 192;
 constexpr float kRescaleLog2 = 8.f;  // rescale O only when the max grows by more
 
 // Shared memory (SW128 regions are 1024-byte aligned).
 struct UmmaSmem {
-    // per stage: K half 0, K half 1, V half 0, V half 1; each [64 pos][64 dims] bf16
+    // per stage: K half 0, K half 1, V half 0, V half 1; each [128 pos][64 dims] bf16
     alignas(1024) uint8_t kv[NST][4][UN * 128];
-    alignas(1024) uint8_t q[2][UM * 128];           // two 64-dim atoms of [128 rows][64]
-    alignas(1024) uint8_t p[2][UM * 128];           // P_hi, P_lo: [128 rows][64 pos]
     uint64_t kv_full[NST];
     uint64_t kv_empty[NST];
     uint64_t q_full;       // softmax warps wrote the item's Q tile
     uint64_t q_free;       // the item's last QK MMA is done with Q
     uint64_t s_full[2];
-    uint64_t s_free[2];
-    uint64_t p_full;       // softmax warps wrote P for the tile
-    uint64_t o_done;       // PV of the tile finished (P buffer free, O readable)
+    uint64_t p_full[2];    // softmax warps wrote P into buffer b
+    uint64_t o_done[2];    // the PV reading P buffer b finished (and every MMA before it)
     uint64_t fin;          // every MMA this CTA issued has completed
     uint32_t tmem_base;
-    volatile uint32_t stage_tile[NST];
     volatile int abort_flag;
 };
 
@@ -84,23 +83,6 @@ __device__ __forceinline__ bool uwait(UmmaSmem &sm, uint64_t *bar, uint32_t pari
     set_flag(flags + 1, site);
     sm.abort_flag = 1;
     return false;
-}
-
-__device__ __forceinline__ bool utag(UmmaSmem &sm, int stage, uint32_t T, uint32_t *flags)
-{
-    const long long t0 = clock64();
-    while (sm.stage_tile[stage] != T) {
-        if (sm.abort_flag)
-            return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
-            set_flag(flags, kDevTimeout);
-            set_flag(flags + 1, kWaitTag);
-            sm.abort_flag = 1;
-            return false;
-        }
-        __nanosleep(32);
-    }
-    return true;
 }
 
 // ---- tcgen05 / TMA wrappers ------------------------------------------------
@@ -138,6 +120,18 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+// O += A B with A read from tensor memory (rows = lanes, K along columns,
+// two bf16 per 32-bit column).
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t *bar)
@@ -228,7 +222,6 @@ __device__ __forceinline__ void umma_producer(const UmmaArgs &a, UmmaSmem &sm)
                 const int st = T % NST;
                 if (!uwait(sm, &sm.kv_empty[st], ((T / NST) & 1u) ^ 1u, p.flags, kWaitEmpty))
                     break;
-                sm.stage_tile[st] = T;
                 if (page_ok) {
                     mbar_arrive_expect_tx(&sm.kv_full[st], 4u * UN * 128u);
                     const int y = row0 + t0;
@@ -254,106 +247,149 @@ __device__ __forceinline__ void umma_producer(const UmmaArgs &a, UmmaSmem &sm)
     }
 }
 
-// The whole MMA warp runs this (lane 0 issues; all lanes zero V tails).
-__device__ __forceinline__ void umma_issuer(const UmmaArgs &a, UmmaSmem &sm, int lane)
+// Tensor-memory columns (448 used of 512):
+//   [0, 256)    two S buffers of 128 fp32 columns.  Once the softmax has read
+//               the 32 columns of S(t) for positions 32c..32c+31, it writes
+//               P_hi of those positions (16 columns of bf16 pairs) and P_lo
+//               (16 more) over them; PV(t) reads them there, and QK(t+2)
+//               overwrites the buffer only after PV(t) in the MMA's issue
+//               order.  S and P are thus both double-buffered.
+//   [256, 384)  O, fp32
+//   [384, 448)  Q, the row's 128 query dims as bf16 pairs
+constexpr uint32_t kColSP = 0;
+constexpr uint32_t kColO = 256;
+constexpr uint32_t kColQ = 384;
+constexpr uint32_t kTmemCols = 512;
+
+// Column of the P part (0: hi, 1: lo) holding positions 16s..16s+15.
+__host__ __device__ constexpr uint32_t p_col(int s, int part)
+{
+    return (uint32_t)(32 * (s >> 1) + 16 * part + 8 * (s & 1));
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// One lane runs this: the ring's only consumer, in order, so its parity
+// waits are unambiguous.  It does as little as possible between MMA batches:
+// the tensor pipe takes a tcgen05.mma about every 100 cycles and idles
+// whenever this thread does anything else.
+// MR is the MMA's M: 128, or 64 for row blocks of at most 64 rows (their
+// accumulator rows sit in lanes m % 16 + 32 * (m / 16) of tensor memory).
+template <int MR>
+__device__ __forceinline__ void umma_issuer(const UmmaArgs &a, UmmaSmem &sm)
 {
     const AttnParams &p = a.p;
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t tS[2] = {tmem, tmem + UN};
-    const uint32_t tO = tmem + 2 * UN;
-    constexpr uint32_t idQK = f16_idesc(UM, UN, 0, 0);
-    constexpr uint32_t idPV = f16_idesc(UM, UD, 0, 1);
-    const uint32_t qa = smem_addr(sm.q[0]);
-    const uint32_t pa[2] = {smem_addr(sm.p[0]), smem_addr(sm.p[1])};
+    constexpr uint32_t idQK = f16_idesc(MR, UN, 0, 0);
+    constexpr uint32_t idPV = f16_idesc(MR, UD, 0, 1);
+    const uint32_t kv0 = smem_addr(sm.kv[0][0]);
+    constexpr uint32_t kHalf = UN * 128;          // one [UN][64] bf16 box
+    constexpr uint32_t kStageBytes = 4 * kHalf;
 
     ItemCursor cur;
     cur.init();
     WorkItem it;
-    uint32_t T0 = 0, j = 0, tt = 0;  // tt: tiles seen by this CTA (S buffer / P phases)
+    uint32_t T0 = 0, j = 0;
+    bool ok = true;
     for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
         const int ntiles = (it.key1 - it.key0 + UN - 1) / UN;
-        bool ok = uwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
+        ok = ok && uwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
         tc_fence_after();
-        // S(t) for t = 0, then per t: S(t+1), then O += P(t) V(t)
-        auto issue_qk = [&](int t) -> bool {
-            const uint32_t T = T0 + t;
+        auto issue_qk = [&](int t) {
+            const uint32_t T = T0 + t;  // CTA-wide tile count (S / P buffer phases too)
             const int st = T % NST;
-            const uint32_t u = tt + t;  // CTA-wide tile count
-            bool good = utag(sm, st, T, p.flags) && uwait(sm, &sm.kv_full[st], (T / NST) & 1u, p.flags, kWaitFull);
-            good = good && uwait(sm, &sm.s_free[u & 1], ((u >> 1) & 1u) ^ 1u, p.flags, kWaitFree);
+            ok = ok && uwait(sm, &sm.kv_full[st], (T / NST) & 1u, p.flags, kWaitFull);
             tc_fence_after();
+            if (!ok)
+                return;
             // positions past the stream's end: zero those V rows (both halves)
             const int tpos = it.key0 + t * UN;
             const int nvalid = min(UN, it.len - tpos);
-            if (good && nvalid < UN) {
-                for (int r = nvalid + (lane >> 3); r < UN; r += 4) {
-                    const int c = lane & 7;
-                    *reinterpret_cast<uint4 *>(sm.kv[st][2] + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(sm.kv[st][3] + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
-                }
+            if (nvalid < UN) {
+                for (int r = nvalid; r < UN; ++r)
+                    for (int c = 0; c < 8; ++c) {
+                        *reinterpret_cast<uint4 *>(sm.kv[st][2] + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(sm.kv[st][3] + sw128_off(r, c)) = make_uint4(0, 0, 0, 0);
+                    }
                 fence_async_smem();
             }
-            __syncwarp();
-            if (good && lane == 0) {
-                const uint32_t ka = smem_addr(sm.kv[st][0]);
+            const uint32_t ka = kv0 + st * kStageBytes;
 #pragma unroll
-                for (int s = 0; s < UD / 16; ++s) {
-                    const uint32_t off = (uint32_t)((s >> 2) * (UM * 128) + (s & 3) * 32);
-                    const uint32_t koff = (uint32_t)((s >> 2) * (UN * 128) + (s & 3) * 32);
-                    umma_f16(tS[u & 1], sw128_desc(qa + off, 16, 1024), sw128_desc(ka + koff, 16, 1024),
-                             idQK, s > 0);
-                }
-                umma_commit(&sm.s_full[u & 1]);
-                if (t == ntiles - 1)
-                    umma_commit(&sm.q_free);
+            for (int s = 0; s < UD / 16; ++s) {
+                const uint32_t koff = (uint32_t)((s >> 2) * kHalf + (s & 3) * 32);
+                umma_f16_ts(tmem + kColSP + 128 * (T & 1), tmem + kColQ + s * 8,
+                            sw128_desc(ka + koff, 16, 1024), idQK, s > 0);
             }
-            __syncwarp();
-            return good;
+            umma_commit(&sm.s_full[T & 1]);
+            if (t == ntiles - 1)
+                umma_commit(&sm.q_free);
         };
-        if (ok)
-            ok = issue_qk(0);
+        issue_qk(0);
         for (int t = 0; t < ntiles; ++t) {
             const uint32_t T = T0 + t;
             const int st = T % NST;
-            const uint32_t u = tt + t;
-            if (ok && t + 1 < ntiles)
-                ok = issue_qk(t + 1);
-            ok = ok && uwait(sm, &sm.p_full, u & 1u, p.flags, kWaitQEmpty);
+            if (t + 1 < ntiles)
+                issue_qk(t + 1);
+            ok = ok && uwait(sm, &sm.p_full[T & 1], (T >> 1) & 1u, p.flags, kWaitQEmpty);
             tc_fence_after();
-            if (ok && lane == 0) {
-                const uint32_t va = smem_addr(sm.kv[st][2]);
+            if (ok) {
+                const uint32_t va = kv0 + st * kStageBytes + 2 * kHalf;
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {
+                    const uint32_t tp = tmem + kColSP + 128 * (T & 1);
 #pragma unroll
-                    for (int s = 0; s < UN / 16; ++s) {
-                        umma_f16(tO, sw128_desc(pa[part] + s * 32, 16, 1024),
-                                 sw128_desc(va + s * 2048, UN * 128, 1024), idPV,
-                                 (t > 0 || part > 0 || s > 0) ? 1u : 0u);
-                    }
+                    for (int s = 0; s < UN / 16; ++s)
+                        umma_f16_ts(tmem + kColO, tp + p_col(s, part),
+                                    sw128_desc(va + s * 2048, kHalf, 1024), idPV,
+                                    (t > 0 || part > 0 || s > 0) ? 1u : 0u);
                 }
-                umma_commit(&sm.o_done);
+                umma_commit(&sm.o_done[T & 1]);
                 umma_commit(&sm.kv_empty[st]);
             }
-            __syncwarp();
         }
         T0 += ntiles;
-        tt += ntiles;
     }
     // every MMA issued by this thread has completed once `fin` flips
-    if (lane == 0) {
-        umma_commit(&sm.fin);
-        (void)mbar_wait(&sm.fin, 0);
-    }
-    __syncwarp();
+    umma_commit(&sm.fin);
+    (void)mbar_wait(&sm.fin, 0);
 }
 
+// Softmax warpgroup: one query row per thread (the row's TMEM lane).  With
+// MR = 64 only lanes 0-15 of each warp hold rows (row 16 * (warp % 4) + lane).
+template <int MR>
 __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, int warp, int lane)
 {
     const AttnParams &p = a.p;
-    const int row = (warp & 3) * 32 + lane;           // TMEM lane == MMA row
+    const int row = MR == 128 ? (warp & 3) * 32 + lane : (warp & 3) * 16 + (lane & 15);
+    const bool lane_rows = MR == 128 || lane < 16;
     const uint32_t lane_base = sm.tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t tS[2] = {lane_base, lane_base + UN};
-    const uint32_t tO = lane_base + 2 * UN;
+    const uint32_t tO = lane_base + kColO;
     const float NEG_INF = -__int_as_float(0x7f800000);
 
     ItemCursor cur;
@@ -361,24 +397,36 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
     WorkItem it;
     uint32_t j = 0, tt = 0;
     for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
-        const int m = it.b * UM + row;
-        const bool live = m < p.M;
+        const int m = it.b * MR + row;
+        const bool live = lane_rows && m < p.M;
         const int lim = row_lim(p, it.len, m);
+        // the first row of the block sees the fewest positions
+        const int lim_lo = row_lim(p, it.len, it.b * MR);
         // --- the row's query into the swizzled Q tile ----------------------
-        bool ok = uwait(sm, &sm.q_free, (j & 1u) ^ 1u, p.flags, kWaitQEmpty);
+        bool ok;
         {
+            // load the row first (overlaps the wait for the previous item's last QK)
             const int mm = min(m, p.M - 1);
             const int wr = mm / p.G;
             const int h = it.kh * p.G + (mm - wr * p.G);
             const uint4 *src = reinterpret_cast<const uint4 *>(
                 p.q + (((size_t)it.s * p.W + wr) * p.Hq + h) * UD);
+            uint32_t qr[2][32];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const uint4 v = live ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-                *reinterpret_cast<uint4 *>(sm.q[c >> 3] + sw128_off(row, c & 7)) = v;
+                qr[c >> 3][(c & 7) * 4 + 0] = v.x;
+                qr[c >> 3][(c & 7) * 4 + 1] = v.y;
+                qr[c >> 3][(c & 7) * 4 + 2] = v.z;
+                qr[c >> 3][(c & 7) * 4 + 3] = v.w;
             }
+            ok = uwait(sm, &sm.q_free, (j & 1u) ^ 1u, p.flags, kWaitQEmpty);
+            tc_fence_after();
+            tmem_st32(lane_base + kColQ, qr[0]);
+            tmem_st32(lane_base + kColQ + 32, qr[1]);
+            tmem_wait_st();
         }
-        fence_async_smem();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0)
             mbar_arrive(&sm.q_full);
@@ -388,43 +436,49 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
         for (int t = 0; t < ntiles; ++t) {
             const uint32_t u = tt + t;
             const int tpos = it.key0 + t * UN;
+            const uint32_t tS = lane_base + kColSP + 128 * (u & 1);
             ok = uwait(sm, &sm.s_full[u & 1], (u >> 1) & 1u, p.flags, kWaitFull) && ok;
             tc_fence_after();
-            float s[UN];
-#pragma unroll
-            for (int c = 0; c < UN / 16; ++c) {
-                uint32_t r[16];
-                tmem_ld16(tS[u & 1] + c * 16, r);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    s[c * 16 + e] = __uint_as_float(r[e]);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sm.s_free[u & 1]);
-            // masked, log2-scaled scores and the tile max
+            // a tile every row of the block sees whole needs no mask; in a
+            // partial tile a row sees positions [tpos, vis_end)
+            const bool whole = tpos + UN <= lim_lo && tpos + UN <= it.key1;
+            const int vis_n = live ? max(0, min(min(lim, it.key1) - tpos, UN)) : 0;
+            const float sl = p.scale_log2;
+            // pass 1: the tile's row max (log2 units)
             float tmax = NEG_INF;
 #pragma unroll
-            for (int e = 0; e < UN; ++e) {
-                const bool vis = live && (tpos + e) < lim && (tpos + e) < it.key1;
-                s[e] = vis ? s[e] * p.scale_log2 : NEG_INF;
-                tmax = fmaxf(tmax, s[e]);
+            for (int c = 0; c < UN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tS + 32 * c, r);
+                tmem_wait_ld();
+                float m0 = NEG_INF, m1 = NEG_INF;
+                if (whole) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        m0 = fmaxf(m0, __uint_as_float(r[e]));
+                        m1 = fmaxf(m1, __uint_as_float(r[e + 1]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        m0 = fmaxf(m0, 32 * c + e < vis_n ? __uint_as_float(r[e]) : NEG_INF);
+                        m1 = fmaxf(m1, 32 * c + e + 1 < vis_n ? __uint_as_float(r[e + 1]) : NEG_INF);
+                    }
+                }
+                tmax = fmaxf(tmax, fmaxf(m0, m1));
             }
+            tmax = (live && tmax != NEG_INF) ? tmax * sl : NEG_INF;
             // a new reference max only when the row max grows by more than 2^8
             const bool grow = tmax > m_run + kRescaleLog2 || (m_run == NEG_INF && tmax != NEG_INF);
             const float m_new = grow ? tmax : m_run;
             const float m_use = m_new == NEG_INF ? 0.f : m_new;
             const float alpha = fast_exp2(m_run - m_use);   // 0 when m_run is -inf
-            // P buffer and O: wait for the previous tile's PV
-            if (t > 0)
-                ok = uwait(sm, &sm.o_done, (u - 1) & 1u, p.flags, kWaitEmpty) && ok;
-            tc_fence_after();
-            // tcgen05.ld/st are warp-collective: rescale when any row of the
-            // warp needs it, by 1 in the rows that do not
             const bool need = grow && t > 0 && m_run != NEG_INF;
-            if (__any_sync(0xffffffffu, need)) {
+            if (__any_sync(0xffffffffu, need)) {   // warp-collective TMEM traffic
+                // S(u) is in, so PV(u - 2) is done (MMAs complete in issue
+                // order): this wait for PV(u - 1) cannot alias an older phase
+                ok = uwait(sm, &sm.o_done[(u - 1) & 1], ((u - 1) >> 1) & 1u, p.flags, kWaitEmpty) && ok;
+                tc_fence_after();
                 const float f = need ? alpha : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < UD / 16; ++c) {
@@ -441,36 +495,50 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
             if (grow)
                 l_run *= alpha;
             m_run = m_new;
-            // P = exp2(s - m) as hi + lo bf16 parts, into the swizzled P tiles
-            float lsum = 0.f;
+            // pass 2: P = exp2(s * scale - m) as hi + lo bf16 parts, written over
+            // the S chunk just read (hi to columns 32c..32c+15, lo after it)
+            float lsum0 = 0.f, lsum1 = 0.f;
+            const float neg_m = -m_use;
 #pragma unroll
-            for (int c = 0; c < UN / 8; ++c) {
-                uint32_t hi[4], lo[4];
+            for (int c = 0; c < UN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tS + 32 * c, r);
+                tmem_wait_ld();
+                uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = fast_exp2(s[c * 8 + 2 * e] - m_use);
-                    const float p1 = fast_exp2(s[c * 8 + 2 * e + 1] - m_use);
-                    lsum += p0 + p1;
-                    hi[e] = pack_bf16(p0, p1);
-                    const float h0 = __uint_as_float(hi[e] << 16);
-                    const float h1 = __uint_as_float(hi[e] & 0xffff0000u);
-                    lo[e] = pack_bf16(p0 - h0, p1 - h1);
+                for (int e = 0; e < 16; ++e) {
+                    float x0 = fmaf(__uint_as_float(r[2 * e]), sl, neg_m);
+                    float x1 = fmaf(__uint_as_float(r[2 * e + 1]), sl, neg_m);
+                    if (!whole) {
+                        x0 = 32 * c + 2 * e < vis_n ? x0 : NEG_INF;
+                        x1 = 32 * c + 2 * e + 1 < vis_n ? x1 : NEG_INF;
+                    }
+                    const float p0 = fast_exp2(x0);
+                    const float p1 = fast_exp2(x1);
+                    lsum0 += p0;
+                    lsum1 += p1;
+                    // P = hi + lo, both bf16 by truncation (upper 16 bits):
+                    // |p - hi - lo| < 2^-14 p.  Packed with byte permutes.
+                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                    hi[e] = __byte_perm(b0, b1, 0x7632);
+                    const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
+                    const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+                    lo[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
                 }
-                *reinterpret_cast<uint4 *>(sm.p[0] + sw128_off(row, c)) =
-                    make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(sm.p[1] + sw128_off(row, c)) =
-                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                tmem_st16(tS + 32 * c, hi);
+                tmem_st16(tS + 32 * c + 16, lo);
             }
+            const float lsum = lsum0 + lsum1;
+            tmem_wait_st();
             l_run += lsum;
-            fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&sm.p_full);
+                mbar_arrive(&sm.p_full[u & 1]);
         }
         // --- the item's last PV, then the row's result ----------------------
         const uint32_t ulast = tt + ntiles - 1;
-        ok = uwait(sm, &sm.o_done, ulast & 1u, p.flags, kWaitEmpty) && ok;
+        ok = uwait(sm, &sm.o_done[ulast & 1], (ulast >> 1) & 1u, p.flags, kWaitEmpty) && ok;
         tc_fence_after();
         const bool write = live && ok && !sm.abort_flag;
         float *dst = nullptr;
@@ -482,7 +550,8 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
                 dst = p.out + (((size_t)it.s * p.W + wr) * p.Hq + h) * UD;
                 sc = 1.f / l_run;
             } else {
-                float *slot = p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(p.RB * (UD + 2));
+                float *slot =
+                    p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(p.RB * (UD + 2));
                 dst = slot + (size_t)row * UD;
                 slot[(size_t)p.RB * UD + row] = m_run;
                 slot[(size_t)p.RB * UD + p.RB + row] = l_run;
@@ -506,6 +575,7 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
     }
 }
 
+template <int MR>
 __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid_constant__ UmmaArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -517,23 +587,21 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
         for (int s = 0; s < NST; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
-            sm.stage_tile[s] = 0xffffffffu;
         }
         mbar_init(&sm.q_full, 4);
         mbar_init(&sm.q_free, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.s_full[s], 1);
-            mbar_init(&sm.s_free[s], 4);
+            mbar_init(&sm.p_full[s], 4);
+            mbar_init(&sm.o_done[s], 1);
         }
-        mbar_init(&sm.p_full, 4);
-        mbar_init(&sm.o_done, 1);
         mbar_init(&sm.fin, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {  // TMEM: 2 S buffers (64 columns each) + O (128 columns)
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
-                         smem_addr(&sm.tmem_base))
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&sm.tmem_base)), "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -546,15 +614,18 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
             umma_producer(a, sm);
         __syncwarp();
     } else if (warp == 1) {
-        umma_issuer(a, sm, lane);
+        if (lane == 0)
+            umma_issuer<MR>(a, sm);
+        __syncwarp();
     } else {
-        umma_softmax(a, sm, warp, lane);
+        umma_softmax<MR>(a, sm, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(sm.tmem_base)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sm.tmem_base),
+                     "r"(kTmemCols)
                      : "memory");
     }
 }
@@ -598,9 +669,11 @@ bool make_pool_map(CUtensorMap *map, const void *pool, const AttnParams &p)
 
 }  // namespace
 
-int umma_rows() { return UM; }
+// Rows of a row block.  (An M = 64 MMA costs about as much time as M = 128
+// on this hardware, so small row counts are padded to 128.)
+int umma_rows(int64_t) { return UM; }
 
-bool umma_supported(int D, int P) { return D == UD && P % UN == 0; }
+bool umma_supported(int D, int P) { return D == UD && P % UN == 0; }  // tiles stay inside a page
 
 cudaError_t launch_attn_umma(const AttnParams &p, int grid, cudaStream_t stream)
 {
@@ -616,13 +689,18 @@ cudaError_t launch_attn_umma(const AttnParams &p, int grid, cudaStream_t stream)
     if (dev < 0 || dev >= kMaxDevices)
         return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(attn_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kUmmaSmemBytes);
-        if (e != cudaSuccess)
-            return e;
+        for (auto fn : {attn_umma_kernel<64>, attn_umma_kernel<128>}) {
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kUmmaSmemBytes);
+            if (e != cudaSuccess)
+                return e;
+        }
         configured[dev] = true;
     }
-    attn_umma_kernel<<<grid, kUmmaThreads, kUmmaSmemBytes, stream>>>(a);
+    if (p.RB == 64)
+        attn_umma_kernel<64><<<grid, kUmmaThreads, kUmmaSmemBytes, stream>>>(a);
+    else
+        attn_umma_kernel<128><<<grid, kUmmaThreads, kUmmaSmemBytes, stream>>>(a);
     return cudaGetLastError();
 }
 

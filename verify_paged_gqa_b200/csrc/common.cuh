@@ -93,10 +93,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete; false after the
-// time limit (the caller records kDevTimeout and winds down).
+// time limit (the caller records kDevTimeout and winds down).  A phase that
+// has already completed costs one non-blocking test.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
+    if (mbar_test_wait(bar, parity))
+        return true;
     if (mbar_try_wait(bar, parity))
         return true;
     const long long t0 = clock64();

@@ -28,8 +28,8 @@ cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream)
 template <int D>
 cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream);
 
-// Tensor-core partial kernel (tcgen05): row blocks of umma_rows() rows.
-int umma_rows();
+// Tensor-core partial kernel (tcgen05): row blocks of umma_rows(M) rows.
+int umma_rows(int64_t M);
 bool umma_supported(int D, int P);
 cudaError_t launch_attn_umma(const AttnParams &p, int grid, cudaStream_t stream);
 

@@ -122,7 +122,7 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     // More than one CUDA-core row block of rows sharing a KV head: a dense
     // QK^T / PV tile for the tensor cores.
     plan->umma = M > kSimtRows && umma_supported(p.D, p.P);
-    p.RB = plan->umma ? umma_rows() : kSimtRows;
+    p.RB = plan->umma ? umma_rows(M) : kSimtRows;
     p.n_rblk = static_cast<int32_t>((M + p.RB - 1) / p.RB);
 
     const int pages_max = (st->max_len + p.P - 1) / p.P;
