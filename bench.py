@@ -25,6 +25,10 @@ With N > 1 (torchrun), every rank runs its own replica of the workload on
 its own GPU (the streams are independent; there is no exchange step):
 weak scaling, value = all ranks' bytes / the slowest rank's time.
 --impl reference times the oracle (rank 0 only) on per-step samples.
+
+The default run also times the draft-verify workload (4 streams at 131,072
+positions, 4 KV / 32 query heads, 8-row windows) the same way and reports its
+verify tokens/s (window rows per second) under "verify" (--no-verify skips).
 """
 from __future__ import annotations
 
@@ -53,6 +57,26 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the workload's dominant kernel, from the ncu capture
+    summarised in profiles/traffic.json -- or None when the kernel's sources have
+    changed since that capture (the hash no longer matches) or there is none."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[workload]
+        h = hashlib.sha256()
+        for name in rec["files"]:
+            with open(os.path.join(ROOT, name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != rec["source_hash"]:
+            return None
+        return int(rec["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def kv_bytes(lens, hkv, d):
@@ -281,26 +305,23 @@ def oracle_sample(wl_name, n_units, threads, device_kv=None):
     n0 = int(lens[0])
     q, k_lin, v_lin = _oracle_inputs(wl_name, device_kv)
     Hq = w.n_q_heads
-    units = [(0, r, h) for r in range(w.rows) for h in range(Hq)][:n_units]
-    units = np.array(units, dtype=np.int32)
+    base = [(0, r, h) for r in range(w.rows) for h in range(Hq)]
+    units = np.array([base[k % len(base)] for k in range(n_units)], dtype=np.int32)
     t0 = time.perf_counter()
     oracle.attend(q, k_lin, v_lin, lens[:1], w.rows, w.group, w.scale, units=units,
                   threads=threads)
     dt = time.perf_counter() - t0
     per_unit = w.head_dim * 2 * 2 / w.group          # one query head's share of a K/V row
     nbytes = sum((n0 - w.rows + int(r) + 1) * per_unit for _, r, _ in units)
-    desc = (f"{len(units)} (stream, row, query head) units of stream 0 at {n0} positions, "
-            f"fp64, {threads} threads")
+    desc = (f"{len(units)} (stream, row, query head) output rows of stream 0 at {n0} positions "
+            f"(the stream's {len(base)} rows, repeated), fp64, {threads} threads")
     return dt, nbytes, desc
 
 
 def cpu_baseline(wl_name, device_kv, budget_s=12.0):
     threads = os.cpu_count() or 1
-    import synth
-    w = synth.WORKLOADS[wl_name]
-    total_units = w.rows * w.n_q_heads
-    dt1, _, _ = oracle_sample(wl_name, min(threads, total_units), threads, device_kv)
-    n = int(min(total_units, max(1, budget_s / max(dt1, 1e-3) * min(threads, total_units))))
+    dt1, _, _ = oracle_sample(wl_name, threads, threads, device_kv)
+    n = int(max(threads, budget_s / max(dt1, 1e-3) * threads))
     dt, nbytes, desc = oracle_sample(wl_name, n, threads, device_kv)
     return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": desc, "seconds": round(dt, 3)}
@@ -315,8 +336,8 @@ def run_reference(args):
     threads = os.cpu_count() or 1
     budget = 150.0
     per_step = budget / max(1, args.steps + args.warmup)
-    dt1, _, _ = oracle_sample(args.workload, min(threads, w.rows * w.n_q_heads), threads)
-    n_units = int(max(1, min(w.rows * w.n_q_heads, per_step / max(dt1, 1e-3) * threads)))
+    dt1, _, _ = oracle_sample(args.workload, threads, threads)
+    n_units = int(max(1, per_step / max(dt1, 1e-3) * threads))
     for _ in range(args.warmup):
         oracle_sample(args.workload, n_units, threads)
     secs, nbytes = 0.0, 0.0
@@ -357,6 +378,7 @@ def main():
     ap.add_argument("--workload", default="decode_12x40k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-verify", action="store_true", help="skip the verify-workload measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -387,6 +409,30 @@ def main():
     wl.check_flags()
     e2e_ms, h2d, d2h = time_e2e(wl, args.steps, args.warmup, barrier)
     wl.check_flags()
+    bytes_per_step, rows_per_step = wl.bytes_per_step, wl.rows_per_step
+
+    # the metric's second half: verify tokens/s on the draft-verify workload
+    secondary = None
+    if args.workload == "decode_12x40k" and not args.no_verify:
+        del wl
+        torch.cuda.empty_cache()
+        vw = Workload("verify_4x131k", f"cuda:{local}")
+        v_total, v_attn = time_steps(vw, args.steps, args.warmup, barrier)
+        vw.check_flags()
+        v_step = v_total / args.steps
+        if dist is not None:
+            t = torch.tensor([v_step, v_attn], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            v_step, v_attn = t.tolist()
+        v_ach = vw.bytes_per_step / (v_attn * 1e-3) / 1e9
+        peak_v, _ = hbm_peak()
+        secondary = {"workload": "verify_4x131k", "verify_tokens_per_s": world * vw.rows_per_step / (v_step * 1e-3),
+                     "kv_gbs": world * vw.bytes_per_step / (v_step * 1e-3) / 1e9, "ms_per_step": v_step,
+                     "attn_ms": v_attn, "roofline_frac": v_ach / peak_v,
+                     "traffic": recorded_traffic("verify_4x131k"),
+                     "gpu_launches": 3 * args.steps, "config": workload_config("verify_4x131k")}
+        del vw
+        torch.cuda.empty_cache()
 
     ms_step = total_ms / args.steps
     e2e_step = e2e_ms / args.steps
@@ -394,28 +440,32 @@ def main():
         t = torch.tensor([ms_step, e2e_step, attn_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step, e2e_step, attn_ms = t.tolist()
-    value = world * wl.bytes_per_step / (ms_step * 1e-3) / 1e9
-    e2e_value = world * wl.bytes_per_step / (e2e_step * 1e-3) / 1e9
+    value = world * bytes_per_step / (ms_step * 1e-3) / 1e9
+    e2e_value = world * bytes_per_step / (e2e_step * 1e-3) / 1e9
     peak, src = hbm_peak()
-    achieved = wl.bytes_per_step / (attn_ms * 1e-3) / 1e9
+    achieved = bytes_per_step / (attn_ms * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(args.workload),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
                      "kernel": "attention call (partial + merge)", "peak_source": src},
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 3 * args.steps,
         "clocks": sampler.summary(),
-        "rows_per_s": world * wl.rows_per_step / (ms_step * 1e-3),
+        "rows_per_s": world * rows_per_step / (ms_step * 1e-3),
         "attn_ms": attn_ms,
     }
+    if secondary is not None:
+        line["verify"] = secondary
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth
-        k, v = synth.kv_rows_torch(wl.w, 0, int(wl.lens_np[0]), f"cuda:{local}")
+        w0 = synth.WORKLOADS[args.workload]
+        n0 = int(synth.stream_lens(w0)[0])
+        k, v = synth.kv_rows_torch(w0, 0, n0, f"cuda:{local}")
         line["cpu_baseline"] = cpu_baseline(args.workload, (k, v))
     if dist is not None:
         dist.barrier()
