@@ -149,3 +149,24 @@ def test_workspace_too_small_is_refused():
     with pytest.raises(tf.TFError) as e:
         dc.attend(ws=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
     assert e.value.status == tf.TF_ENOSPACE
+
+
+@pytest.mark.parametrize("d,G,W", [(128, 8, 8), (128, 4, 3), (512, 8, 4), (512, 4, 8),
+                                   (128, 4, 1), (128, 4, 100)])
+def test_parity_growing_scores(d, G, W):
+    """K rows scaled up along the context: every row's max keeps growing past
+    the kernels' rescale margin, so running maxima move and O is rescaled
+    many times inside one chunk."""
+    w = small_workload(d, G, 512, W, seed=8000 + d + 10 * G + W)
+    case = synth.make_case(w, lens=[3000, 1300 + W], rows=W)
+    for s, n in enumerate(case.lens):
+        ramp = (1.0 + 14.0 * np.arange(n) / n).astype(np.float32)[:, None, None]
+        k = synth.f32_from_bf16(case.k_lin[s]) * ramp
+        case.k_lin[s] = synth.bf16_from_f32(k)
+    dc = DeviceCase(case)
+    out = dc.attend()
+    torch.cuda.synchronize()
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, W, w.group, w.scale,
+                        threads=8)
+    assert torch.isfinite(out).all()
+    assert max_abs(out, ref) <= TOL

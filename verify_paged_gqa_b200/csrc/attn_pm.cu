@@ -1,0 +1,750 @@
+// attn_pm.cu -- split-context paged attention on the 5th-generation tensor
+// cores with the key positions on the MMA's M dimension ("position-major"),
+// for row blocks of up to 64 query rows: draft-verify windows, decode at
+// GQA 8, and every head dim 512 case.
+//
+// TensorFold #1620 ("Kolibri-1's full layers take their K/V from pages of
+// the core pool"), opening comment, "Reads": decode, verify and prompt rows
+// attend over keys read through the page table; TensorFold #2730 ("an
+// eight-row verify window"), "What this changes": a window holds up to eight
+// rows.  The M = G * W rows of one (stream, KV head) share every K and V row.
+// With rows on the MMA's M a 64-row verify block would be padded to 128,
+// wasting half the tensor and softmax work, so this kernel computes the
+// transposed products instead:
+//
+//   S^T[pos][r]  = sum_d K[pos][d] Q[r][d]       M = 128 positions, N = NR rows
+//   O^T[d][r]   += sum_pos V[pos][d] P[r][pos]   M = 128 dims, N = 2 NR
+//
+// M is always full, and one softmax thread owns one key position of the
+// tile: its tensor-memory lane of S^T.  P is fed to the PV MMA from shared
+// memory as two bf16 parts (P = hi + lo, each the truncated upper half of a
+// float, so the product keeps about 15 bits of every probability); hi and lo
+// sit side by side along N and land in separate O^T columns that the
+// epilogue adds.
+//
+// One persistent CTA per SM, six warps:
+//   warp 0     producer (one lane): per tile, the K units of the next tile,
+//              then the V units of this one (a unit is 128 positions x 128
+//              dims, two 64-dim TMA boxes with 128-byte swizzle) into a ring;
+//              page ids are read two tiles ahead.
+//   warp 1     MMA issuer (one lane): S^T(t+1) = K Q^T before O^T += V^T P^T(t),
+//              so the softmax of one tile overlaps the MMAs of the next.
+//              Owns the tensor-memory allocation.
+//   warps 2-5  softmax, one key position per thread: write the block's query
+//              rows into the Q tile at each item's start; per tile, read the
+//              position's scores for all rows, check them against each row's
+//              reference max (a block-wide vote; the reference moves only
+//              when some row's max grows by more than 2^8, and then O^T is
+//              rescaled), write P^T, and keep per-thread row sums.  At the
+//              item's end the sums are reduced across the block and the rows
+//              are normalised and stored, or left as partials for the merge.
+#include "launch.cuh"
+#include "plan.cuh"
+#include "umma.cuh"
+
+namespace tfp {
+
+namespace {
+
+constexpr int PT = 128;                  // key positions per tile (the MMA's M)
+constexpr uint32_t kBox = 16384;         // one [128 positions][64 dims] bf16 SW128 box
+constexpr uint32_t kUnit = 2 * kBox;     // one ring unit: 128 positions x 128 dims
+constexpr float kRescaleLog2 = 8.f;      // move a row's reference max only past this growth
+constexpr uint32_t kSmemCap = 232448;    // dynamic shared memory per block
+
+template <int D, int NR>
+struct PmCfg {
+    static constexpr int DB = D / 128;                         // units per K (or V) tile
+    static constexpr uint32_t kQBytes = (uint32_t)NR * D * 2;  // Q tile, 64-dim SW128 boxes
+    static constexpr uint32_t kPBytes = (uint32_t)PT * 2 * NR * 2;  // P^T: [128 pos][2 NR] bf16
+    // tensor memory: two S^T buffers of NR columns, then DB O^T blocks of 2 NR
+    static constexpr uint32_t kColS = 0;
+    static constexpr uint32_t kColO = 2 * NR;
+    static constexpr uint32_t kCols = 2 * NR + DB * 2 * NR;
+    static constexpr uint32_t kTmemCols =
+        kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
+    static constexpr uint32_t kSmall = 48 * NR + 512;  // per-row arrays and barriers
+    static constexpr int kFit = (int)((kSmemCap - 1024 - kQBytes - 2 * kPBytes - kSmall) / kUnit);
+    static constexpr int NU = kFit > 6 ? 6 : kFit;     // ring units
+    static_assert(kCols <= 512, "tensor memory");
+    static_assert(NU >= 2, "ring");
+    static_assert(NR == 32 || NR == 64, "row block");
+    static constexpr int kSoftThreads = 4 * NR;        // 32 rows per softmax thread
+    static constexpr int kThreads = 64 + kSoftThreads; // + producer and MMA warps
+};
+
+template <int D, int NR>
+struct PmSmem {
+    using C = PmCfg<D, NR>;
+    alignas(1024) uint8_t ring[C::NU][kUnit];
+    alignas(1024) uint8_t q[C::kQBytes];
+    alignas(1024) uint8_t pt[2][C::kPBytes];
+    alignas(16) float mref[NR];   // row reference max, log2 units; -inf while the row saw nothing
+    alignas(16) float negm[NR];   // -mref, or +inf while mref is -inf (forces a new reference)
+    alignas(16) float alpha[NR];  // factor of the last reference change
+    alignas(16) float lsum[NR];   // row sums (inverted for a finished row block)
+    alignas(16) float red[4][NR];
+    long long rowoff[2][NR];      // output offset of row r (by item parity); -1 past M
+    uint64_t full[C::NU];
+    uint64_t empty[C::NU];
+    uint64_t q_full;      // the softmax warps wrote the item's Q tile
+    uint64_t q_free;      // the item's last QK MMA is done with the Q tile
+    uint64_t s_full[2];   // S^T(t) is in tensor memory
+    uint64_t p_full[2];   // the softmax warps wrote P^T(t)
+    uint64_t o_done[2];   // the PV reading P^T buffer b (and every MMA before it) completed
+    uint64_t fin;
+    uint32_t tmem_base;
+    volatile int abort_flag;
+};
+
+template <int D, int NR>
+constexpr size_t pm_smem_bytes()
+{
+    return sizeof(PmSmem<D, NR>) + 1024;  // + alignment slack
+}
+
+static_assert(pm_smem_bytes<128, 32>() <= kSmemCap, "smem");
+static_assert(pm_smem_bytes<128, 64>() <= kSmemCap, "smem");
+static_assert(pm_smem_bytes<512, 32>() <= kSmemCap, "smem");
+
+struct PmArgs {
+    AttnParams p;
+    CUtensorMap kmap;
+    CUtensorMap vmap;
+};
+
+template <class Sm>
+__device__ __forceinline__ bool pwait(Sm &sm, uint64_t *bar, uint32_t parity, uint32_t *flags,
+                                      uint32_t site)
+{
+    if (sm.abort_flag)
+        return false;
+    if (mbar_wait(bar, parity))
+        return true;
+    set_flag(flags, kDevTimeout);
+    set_flag(flags + 1, site);
+    sm.abort_flag = 1;
+    return false;
+}
+
+// OR of `pred` over the NT softmax threads (named barrier 1).
+template <int NT>
+__device__ __forceinline__ bool block_any(bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, %2, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "n"(NT)
+        : "memory");
+    return r != 0;
+}
+
+// Reduces v[i] (one value per row, N rows) across the warp: lane l ends up
+// holding the reduction of rows [l * N / 32, (l + 1) * N / 32) in v[0 ..].
+// Each step sends half of the remaining rows to the partner lane.
+template <int N, bool kMax>
+__device__ __forceinline__ void xpose_reduce(float (&v)[N], int lane)
+{
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const int o = 16 >> k;
+        const int n = N >> k;
+        if (n > 1) {
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < n / 2; ++i) {
+                const float send = up ? v[i] : v[i + n / 2];
+                const float keep = up ? v[i + n / 2] : v[i];
+                const float got = __shfl_xor_sync(0xffffffffu, send, o);
+                v[i] = kMax ? fmaxf(keep, got) : keep + got;
+            }
+        }
+    }
+}
+
+// The NR scores of this thread's position (its S^T lane), waited for.
+template <int NR>
+__device__ __forceinline__ void load_scores(uint32_t taddr, float (&x)[NR])
+{
+#pragma unroll
+    for (int c = 0; c < NR / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + 32 * c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            x[32 * c + e] = __uint_as_float(r[e]);
+    }
+}
+
+// ---- producer ----------------------------------------------------------------
+
+// Loads the DB units of one K or V tile (positions [off, off + 128) of a page).
+template <int D, int NR>
+__device__ __forceinline__ bool pm_put_tile(const AttnParams &p, PmSmem<D, NR> &sm, uint32_t &U,
+                                            const CUtensorMap *map, int page, int kh, int off,
+                                            uint64_t pol)
+{
+    using C = PmCfg<D, NR>;
+    const bool page_ok = page >= 0 && page < p.n_pages;
+    if (!page_ok)
+        set_flag(p.flags, kDevBadPage);
+    const int y = ((page_ok ? page : 0) * p.Hkv + kh) * p.P + off;
+#pragma unroll 1
+    for (int kb = 0; kb < C::DB; ++kb) {
+        const int st = (int)(U % C::NU);
+        if (!pwait(sm, &sm.empty[st], ((U / C::NU) & 1u) ^ 1u, p.flags, kWaitEmpty))
+            return false;
+        if (page_ok) {
+            mbar_arrive_expect_tx(&sm.full[st], kUnit);
+            tma_load_2d(sm.ring[st], map, 128 * kb, y, &sm.full[st], pol);
+            tma_load_2d(sm.ring[st] + kBox, map, 128 * kb + 64, y, &sm.full[st], pol);
+        } else {
+            mbar_arrive(&sm.full[st]);
+        }
+        ++U;
+    }
+    return true;
+}
+
+// Unit order per item (the issuer consumes in the same order):
+// K(0), then for each tile t: K(t + 1) if any, V(t).
+template <int D, int NR>
+__device__ __forceinline__ void pm_producer(const PmArgs &a, PmSmem<D, NR> &sm)
+{
+    using C = PmCfg<D, NR>;
+    const AttnParams &p = a.p;
+    const uint64_t pol = l2_evict_first_policy();
+    ItemCursor cur;
+    cur.init();
+    WorkItem it;
+    uint32_t U = 0;
+    bool ok = true;
+    for (int64_t i = blockIdx.x; ok && cur.seek(p, i, it); i += gridDim.x) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
+        int pg0 = __ldg(trow + it.key0 / p.P);
+        int pg1 = n > 1 ? __ldg(trow + (it.key0 + PT) / p.P) : 0;
+        ok = pm_put_tile(p, sm, U, &a.kmap, pg0, it.kh, it.key0 % p.P, pol);
+        for (int t = 0; ok && t < n; ++t) {
+            const int pos = it.key0 + t * PT;
+            const int pg2 = t + 2 < n ? __ldg(trow + (pos + 2 * PT) / p.P) : 0;
+            if (t + 1 < n)
+                ok = pm_put_tile(p, sm, U, &a.kmap, pg1, it.kh, (pos + PT) % p.P, pol);
+            if (ok)
+                ok = pm_put_tile(p, sm, U, &a.vmap, pg0, it.kh, pos % p.P, pol);
+            pg0 = pg1;
+            pg1 = pg2;
+        }
+    }
+    if (!ok || sm.abort_flag) {
+        // let the copies in flight land before the CTA exits
+        const uint32_t nf = U < (uint32_t)C::NU ? U : (uint32_t)C::NU;
+        for (uint32_t k = 1; k <= nf; ++k) {
+            const uint32_t v = U - k;
+            (void)mbar_wait(&sm.full[v % C::NU], (v / C::NU) & 1u);
+        }
+    }
+}
+
+// ---- MMA issuer --------------------------------------------------------------
+
+// S^T = K Q^T for one tile: DB units, 8 MMAs (K = 16 dims) each.
+template <int D, int NR>
+__device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d_tmem,
+                                      uint32_t ring0, uint32_t q0, uint32_t *flags)
+{
+    using C = PmCfg<D, NR>;
+    constexpr uint32_t idQK = f16_idesc(128, NR, 0, 0);
+#pragma unroll 1
+    for (int kb = 0; kb < C::DB; ++kb) {
+        const int st = (int)(U % C::NU);
+        if (!pwait(sm, &sm.full[st], (U / C::NU) & 1u, flags, kWaitFull))
+            return false;
+        tc_fence_after();
+        const uint32_t ka = ring0 + st * kUnit;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const uint32_t koff = (uint32_t)((s >> 2) * kBox + (s & 3) * 32);
+            const uint32_t qoff = (uint32_t)((2 * kb + (s >> 2)) * (NR * 128) + (s & 3) * 32);
+            umma_f16(d_tmem, sw128_desc(ka + koff, 16, 1024), sw128_desc(q0 + qoff, 16, 1024), idQK,
+                     (kb > 0 || s > 0) ? 1u : 0u);
+        }
+        umma_commit(&sm.empty[st]);
+        ++U;
+    }
+    return true;
+}
+
+template <int D, int NR>
+__device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
+{
+    using C = PmCfg<D, NR>;
+    const AttnParams &p = a.p;
+    const uint32_t tmem = sm.tmem_base;
+    constexpr uint32_t idPV = f16_idesc(128, 2 * NR, 1, 1);
+    const uint32_t ring0 = smem_addr(sm.ring[0]);
+    const uint32_t q0 = smem_addr(sm.q);
+    const uint32_t pt0 = smem_addr(sm.pt[0]);
+
+    ItemCursor cur;
+    cur.init();
+    WorkItem it;
+    uint32_t U = 0, T0 = 0, j = 0;
+    bool ok = true;
+    for (int64_t i = blockIdx.x; ok && cur.seek(p, i, it); i += gridDim.x, ++j) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        ok = pwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
+        tc_fence_after();
+        ok = ok && pm_qk(sm, U, tmem + C::kColS + (T0 & 1u) * NR, ring0, q0, p.flags);
+        if (!ok)
+            break;
+        umma_commit(&sm.s_full[T0 & 1u]);
+        if (n == 1)
+            umma_commit(&sm.q_free);
+        for (int t = 0; t < n; ++t) {
+            const uint32_t T = T0 + t;
+            if (t + 1 < n) {
+                ok = pm_qk(sm, U, tmem + C::kColS + ((T + 1) & 1u) * NR, ring0, q0, p.flags);
+                if (!ok)
+                    break;
+                umma_commit(&sm.s_full[(T + 1) & 1u]);
+                if (t + 2 == n)
+                    umma_commit(&sm.q_free);
+            }
+            ok = pwait(sm, &sm.p_full[T & 1u], (T >> 1) & 1u, p.flags, kWaitQEmpty);
+            tc_fence_after();
+            if (!ok)
+                break;
+            const uint32_t pb = pt0 + (T & 1u) * C::kPBytes;
+#pragma unroll 1
+            for (int vb = 0; vb < C::DB; ++vb) {
+                const int st = (int)(U % C::NU);
+                ok = pwait(sm, &sm.full[st], (U / C::NU) & 1u, p.flags, kWaitFull);
+                tc_fence_after();
+                if (!ok)
+                    break;
+                const uint32_t va = ring0 + st * kUnit;
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    umma_f16(tmem + C::kColO + vb * 2 * NR, sw128_desc(va + s * 2048, kBox, 1024),
+                             sw128_desc(pb + s * 2048, kBox, 1024), idPV, (t > 0 || s > 0) ? 1u : 0u);
+                umma_commit(&sm.empty[st]);
+                ++U;
+            }
+            if (!ok)
+                break;
+            umma_commit(&sm.o_done[T & 1u]);
+        }
+        T0 += n;
+    }
+    // every MMA issued by this thread has completed once `fin` flips
+    umma_commit(&sm.fin);
+    (void)mbar_wait(&sm.fin, 0);
+}
+
+// ---- softmax warps -----------------------------------------------------------
+
+// NW = 4 * NR / 32 softmax warps: warp w reads tensor-memory lanes
+// 32 * (w % 4) .. + 31 (tile positions, or O^T dims), and owns the 32 rows
+// [32 h, 32 h + 32) with h = (w - 2) / 4.
+template <int D, int NR>
+__device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, int warp, int lane)
+{
+    using C = PmCfg<D, NR>;
+    constexpr int NT = C::kSoftThreads;
+    const AttnParams &p = a.p;
+    const int wq = warp & 3;             // tensor-memory lane quarter of this warp
+    const int h = (warp - 2) >> 2;       // row half: rows [32 h, 32 h + 32)
+    const int tid = wq * 32 + lane;      // position in the tile; O^T lane (dim within a block)
+    const int st = (warp - 2) * 32 + lane;  // 0 .. NT - 1
+    const uint32_t lane_base = sm.tmem_base + ((uint32_t)(wq * 32) << 16);
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    const float POS_INF = __int_as_float(0x7f800000);
+    const float sl = p.scale_log2;
+    // this thread's row of a P^T buffer (SW128: 8-row groups of 1024 bytes)
+    const uint32_t prow = (uint32_t)((tid >> 3) * 1024 + (tid & 7) * 128);
+    const int sw = tid & 7;
+    const int R0 = 32 * h;               // first row of this thread
+
+    ItemCursor cur;
+    cur.init();
+    WorkItem it;
+    uint32_t j = 0, u0 = 0;
+    bool ok = true;
+    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        // --- the block's query rows into the Q tile; output offsets ---------
+        {
+            constexpr int kPer = NR * D / 8 / NT;  // 16-byte chunks per thread
+            static_assert(kPer % 4 == 0, "Q chunks");
+            if (st < NR) {
+                const int m = it.b * NR + st;
+                long long off = -1;
+                if (m < p.M) {
+                    const int wr = m / p.G;
+                    const int hq = it.kh * p.G + (m - wr * p.G);
+                    off = (((long long)it.s * p.W + wr) * p.Hq + hq) * D;
+                }
+                sm.rowoff[j & 1u][st] = off;
+            }
+            // (already complete in practice: the previous item's last PV,
+            // waited for below, was issued after its last QK)
+            ok = pwait(sm, &sm.q_free, (j & 1u) ^ 1u, p.flags, kWaitQEmpty) && ok;
+#pragma unroll
+            for (int c0 = 0; c0 < kPer; c0 += 4) {
+                uint4 qv[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int f = st + NT * (c0 + c);
+                    const int r = f / (D / 8), k = f % (D / 8);
+                    const int m = it.b * NR + r;
+                    qv[c] = make_uint4(0, 0, 0, 0);
+                    if (m < p.M) {
+                        const int wr = m / p.G;
+                        const int hq = it.kh * p.G + (m - wr * p.G);
+                        qv[c] = __ldg(reinterpret_cast<const uint4 *>(
+                                          p.q + (((size_t)it.s * p.W + wr) * p.Hq + hq) * D) +
+                                      k);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int f = st + NT * (c0 + c);
+                    const int r = f / (D / 8), k = f % (D / 8);
+                    *reinterpret_cast<uint4 *>(sm.q + (k >> 3) * (NR * 128) + sw128_off(r, k & 7)) =
+                        qv[c];
+                }
+            }
+            fence_async_smem();
+            named_barrier(1, NT);
+            if (st == 0)
+                mbar_arrive(&sm.q_full);
+        }
+
+        float l[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+            l[r] = 0.f;
+        // the block's first row sees the fewest positions
+        const int lim_lo = row_lim(p, it.len, it.b * NR);
+        for (int t = 0; t < n; ++t) {
+            const uint32_t u = u0 + t;
+            const int tpos = it.key0 + t * PT;
+            const uint32_t tS = lane_base + C::kColS + (u & 1u) * NR + R0;
+            // a tile every row of the block sees whole needs no mask
+            const bool whole = tpos + PT <= lim_lo && tpos + PT <= it.key1;
+            // rows R0 + r, r >= rvis, see this thread's position
+            const int pos = tpos + tid;
+            const int rvis = (pos >= it.key1 || pos >= it.len)
+                                 ? 32
+                                 : p.G * max(0, pos - (it.len - p.W)) - it.b * NR - R0;
+            ok = pwait(sm, &sm.s_full[u & 1u], (u >> 1) & 1u, p.flags, kWaitFull) && ok;
+            tc_fence_after();
+
+            float x[32];
+            bool slow = t == 0;
+            if (!slow) {
+                load_scores<32>(tS, x);
+                float mx = NEG_INF;
+#pragma unroll
+                for (int r = 0; r < 32; r += 4) {
+                    const float4 nm = *reinterpret_cast<const float4 *>(&sm.negm[R0 + r]);
+                    x[r] = fmaf(x[r], sl, nm.x);
+                    x[r + 1] = fmaf(x[r + 1], sl, nm.y);
+                    x[r + 2] = fmaf(x[r + 2], sl, nm.z);
+                    x[r + 3] = fmaf(x[r + 3], sl, nm.w);
+                }
+                if (!whole) {
+#pragma unroll
+                    for (int r = 0; r < 32; ++r)
+                        x[r] = r >= rvis ? x[r] : NEG_INF;
+                }
+#pragma unroll
+                for (int r = 0; r < 32; ++r)
+                    mx = fmaxf(mx, x[r]);
+                slow = block_any<NT>(mx > kRescaleLog2);
+            }
+            if (slow) {
+                // --- a new reference max for rows whose max grew past it ---
+                float y[32];
+                load_scores<32>(tS, y);
+#pragma unroll
+                for (int r = 0; r < 32; ++r)
+                    y[r] = (whole || r >= rvis) ? y[r] * sl : NEG_INF;
+                xpose_reduce<32, true>(y, lane);
+                sm.red[wq][R0 + lane] = y[0];
+                named_barrier(1, NT);
+                bool moved = false;
+                if (st < NR) {
+                    const float tmax = fmaxf(fmaxf(sm.red[0][st], sm.red[1][st]),
+                                             fmaxf(sm.red[2][st], sm.red[3][st]));
+                    const float m_old = t == 0 ? NEG_INF : sm.mref[st];
+                    const bool grow =
+                        tmax != NEG_INF && (m_old == NEG_INF || tmax > m_old + kRescaleLog2);
+                    const float m_new = grow ? tmax : m_old;
+                    sm.mref[st] = m_new;
+                    sm.negm[st] = m_new == NEG_INF ? POS_INF : -m_new;
+                    sm.alpha[st] = !grow ? 1.f : (m_old == NEG_INF ? 0.f : fast_exp2(m_old - m_new));
+                    moved = t > 0 && grow && m_old != NEG_INF;
+                }
+                moved = block_any<NT>(moved);  // also publishes mref / negm / alpha
+                if (moved) {
+                    // PV(u - 1) must be done before O^T is touched; this warp
+                    // rescales its rows' hi and lo columns of every dim block
+                    ok = pwait(sm, &sm.o_done[(u - 1) & 1u], ((u - 1) >> 1) & 1u, p.flags,
+                               kWaitEmpty) && ok;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < 2 * C::DB; ++c) {
+                        const uint32_t ta =
+                            lane_base + C::kColO + (c >> 1) * 2 * NR + (c & 1) * NR + R0;
+                        uint32_t r[32];
+                        tmem_ld32(ta, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            r[e] = __float_as_uint(__uint_as_float(r[e]) * sm.alpha[R0 + e]);
+                        tmem_st32(ta, r);
+                    }
+                    tmem_wait_st();
+                }
+                load_scores<32>(tS, x);
+#pragma unroll
+                for (int r = 0; r < 32; r += 4) {
+                    const float4 nm = *reinterpret_cast<const float4 *>(&sm.negm[R0 + r]);
+                    const float4 al = *reinterpret_cast<const float4 *>(&sm.alpha[R0 + r]);
+                    x[r] = fmaf(x[r], sl, nm.x);
+                    x[r + 1] = fmaf(x[r + 1], sl, nm.y);
+                    x[r + 2] = fmaf(x[r + 2], sl, nm.z);
+                    x[r + 3] = fmaf(x[r + 3], sl, nm.w);
+                    l[r] *= al.x;
+                    l[r + 1] *= al.y;
+                    l[r + 2] *= al.z;
+                    l[r + 3] *= al.w;
+                }
+                if (!whole) {
+#pragma unroll
+                    for (int r = 0; r < 32; ++r)
+                        x[r] = r >= rvis ? x[r] : NEG_INF;
+                }
+            }
+            // --- V rows past the stream's end: zero them (0 * NaN = NaN) ----
+            const int nvalid = it.len - tpos;
+            if (nvalid < PT) {
+                // the V units of this tile: K(0), then per tile K(t + 1) if any, V(t)
+                uint32_t uv = 2u * C::DB * u0 + C::DB * (2u * t + 1u + (t + 1 < n ? 1u : 0u));
+#pragma unroll 1
+                for (int vb = 0; vb < C::DB; ++vb, ++uv) {
+                    const int sl8 = (int)(uv % C::NU);
+                    ok = pwait(sm, &sm.full[sl8], (uv / C::NU) & 1u, p.flags, kWaitFull) && ok;
+                    if (tid >= nvalid) {
+                        // the NW / 4 threads of a position split the unit's two boxes
+#pragma unroll 1
+                        for (int bx = h; bx < 2; bx += NR / 32) {
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4 *>(sm.ring[sl8] + bx * kBox + sw128_off(tid, c)) =
+                                    make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+            }
+            // --- P^T(u): buffer u & 1 is free once PV(u - 2) completed -----
+            if (u >= 2)
+                ok = pwait(sm, &sm.o_done[u & 1u], ((u - 2) >> 1) & 1u, p.flags, kWaitEmpty) && ok;
+            uint8_t *pr = sm.pt[u & 1u] + prow;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = 8 * g + 2 * e;
+                    const float p0 = fast_exp2(x[r]);
+                    const float p1 = fast_exp2(x[r + 1]);
+                    l[r] += p0;
+                    l[r + 1] += p1;
+                    // P = hi + lo, both bf16 by truncation: |p - hi - lo| < 2^-14 p
+                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                    hw[e] = __byte_perm(b0, b1, 0x7632);
+                    const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
+                    const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+                    lw[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+                }
+                // hi of rows R0 + 8g .. + 7 is 16-byte chunk R0 / 8 + g of the
+                // position's row; lo is chunk (NR + R0) / 8 + g
+                const int ch = R0 / 8 + g, cl = (NR + R0) / 8 + g;
+                *reinterpret_cast<uint4 *>(pr + (ch >> 3) * kBox + (((ch & 7) ^ sw) << 4)) =
+                    make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(pr + (cl >> 3) * kBox + (((cl & 7) ^ sw) << 4)) =
+                    make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.p_full[u & 1u]);
+        }
+
+        // --- the item's last PV, then the rows' results ------------------------
+        const uint32_t ulast = u0 + n - 1;
+        ok = pwait(sm, &sm.o_done[ulast & 1u], (ulast >> 1) & 1u, p.flags, kWaitEmpty) && ok;
+        tc_fence_after();
+        const bool fin = it.nc == 1;
+        xpose_reduce<32, false>(l, lane);
+        sm.red[wq][R0 + lane] = l[0];
+        named_barrier(1, NT);
+        if (st < NR) {
+            const float s = sm.red[0][st] + sm.red[1][st] + sm.red[2][st] + sm.red[3][st];
+            sm.lsum[st] = fin ? 1.f / s : s;
+        }
+        named_barrier(1, NT);
+        const bool write = ok && !sm.abort_flag;
+        float *slot = fin ? nullptr
+                          : p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(NR * (D + 2));
+#pragma unroll 1
+        for (int vb = 0; vb < C::DB; ++vb) {
+            uint32_t hi[32], lo[32];
+            tmem_ld32(lane_base + C::kColO + vb * 2 * NR + R0, hi);
+            tmem_ld32(lane_base + C::kColO + vb * 2 * NR + NR + R0, lo);
+            tmem_wait_ld();
+            if (write) {
+                const int d = 128 * vb + tid;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int r = R0 + e;
+                    const float o = __uint_as_float(hi[e]) + __uint_as_float(lo[e]);
+                    if (fin) {
+                        const long long off = sm.rowoff[j & 1u][r];
+                        if (off >= 0)
+                            p.out[off + d] = o * sm.lsum[r];
+                    } else {
+                        slot[(size_t)r * D + d] = o;
+                    }
+                }
+            }
+        }
+        if (write && !fin && st < NR) {
+            slot[(size_t)NR * D + st] = sm.mref[st];
+            slot[(size_t)NR * D + NR + st] = sm.lsum[st];
+        }
+        tc_fence_before();
+        u0 += n;
+    }
+}
+
+template <int D, int NR>
+__global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
+    attn_pm_kernel(const __grid_constant__ PmArgs a)
+{
+    using C = PmCfg<D, NR>;
+    extern __shared__ uint8_t smem_raw[];
+    PmSmem<D, NR> &sm = *reinterpret_cast<PmSmem<D, NR> *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NU; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.q_full, 1);
+        mbar_init(&sm.q_free, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.p_full[b], C::kSoftThreads / 32);
+            mbar_init(&sm.o_done[b], 1);
+        }
+        mbar_init(&sm.fin, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&sm.tmem_base)), "r"(C::kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == 0) {
+        if (lane == 0)
+            pm_producer<D, NR>(a, sm);
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0)
+            pm_issuer<D, NR>(a, sm);
+        __syncwarp();
+    } else {
+        pm_softmax<D, NR>(a, sm, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sm.tmem_base),
+                     "r"(C::kTmemCols)
+                     : "memory");
+    }
+}
+
+template <int D, int NR>
+cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
+{
+    PmArgs a;
+    a.p = p;
+    if (!make_pool_map(&a.kmap, p.k_pool, p, PT) || !make_pool_map(&a.vmap, p.v_pool, p, PT))
+        return cudaErrorInvalidValue;
+    static bool configured[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    constexpr size_t bytes = pm_smem_bytes<D, NR>();
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(attn_pm_kernel<D, NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)bytes);
+        if (e != cudaSuccess)
+            return e;
+        configured[dev] = true;
+    }
+    attn_pm_kernel<D, NR><<<grid, PmCfg<D, NR>::kThreads, bytes, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Rows per row block, or 0 when this kernel does not take the call: tiles
+// stay inside a page, and blocks of more than 64 rows at head dim 128 go to
+// the row-major tensor-core kernel.
+int pm_rows(const AttnParams &p)
+{
+    if (p.P % PT != 0 || !pool_rows_fit(p))
+        return 0;
+    if (p.D == 128)
+        return p.M <= 32 ? 32 : p.M <= 64 ? 64 : 0;
+    if (p.D == 512)
+        return 32;
+    return 0;
+}
+
+cudaError_t launch_attn_pm(const AttnParams &p, int grid, cudaStream_t stream)
+{
+    if (p.D == 128 && p.RB == 32)
+        return launch_pm<128, 32>(p, grid, stream);
+    if (p.D == 128 && p.RB == 64)
+        return launch_pm<128, 64>(p, grid, stream);
+    if (p.D == 512 && p.RB == 32)
+        return launch_pm<512, 32>(p, grid, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace tfp

@@ -28,9 +28,15 @@ cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream)
 template <int D>
 cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream);
 
-// Tensor-core partial kernel (tcgen05): row blocks of umma_rows(M) rows.
+// Row-major tensor-core partial kernel (tcgen05): row blocks of
+// umma_rows(M) rows on the MMA's M.
 int umma_rows(int64_t M);
-bool umma_supported(int D, int P);
+bool umma_supported(const AttnParams &p);
 cudaError_t launch_attn_umma(const AttnParams &p, int grid, cudaStream_t stream);
+
+// Position-major tensor-core partial kernel: key positions on the MMA's M,
+// row blocks of pm_rows(p) rows (0: not supported for these arguments).
+int pm_rows(const AttnParams &p);
+cudaError_t launch_attn_pm(const AttnParams &p, int grid, cudaStream_t stream);
 
 }  // namespace tfp

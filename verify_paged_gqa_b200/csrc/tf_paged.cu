@@ -56,11 +56,13 @@ int check_pool_streams(const tf_kv_pool *pool, const tf_streams *st)
     return TF_OK;
 }
 
+enum class Kernel { kSimt, kUmma, kPm };
+
 struct Plan {
     AttnParams p;
     int grid;
     size_t ws_bytes;
-    bool umma;  // tensor-core partial kernel (else the CUDA-core one)
+    Kernel kernel;  // which partial kernel runs the call
 };
 
 // Chunk length in pages: the one that minimises the busiest CTA's pages
@@ -120,9 +122,21 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     p.W = rows;
     p.M = static_cast<int32_t>(M);
     // More than one CUDA-core row block of rows sharing a KV head: a dense
-    // QK^T / PV tile for the tensor cores.
-    plan->umma = M > kSimtRows && umma_supported(p.D, p.P);
-    p.RB = plan->umma ? umma_rows(M) : kSimtRows;
+    // QK^T / PV tile for the tensor cores.  Up to 64 rows (128 at head dim
+    // 512 in blocks of 32) go with the positions on the MMA's M; larger
+    // blocks with the rows there.
+    plan->kernel = Kernel::kSimt;
+    p.RB = kSimtRows;
+    if (M > kSimtRows) {
+        const int nr = pm_rows(p);
+        if (nr > 0) {
+            plan->kernel = Kernel::kPm;
+            p.RB = nr;
+        } else if (umma_supported(p)) {
+            plan->kernel = Kernel::kUmma;
+            p.RB = umma_rows(M);
+        }
+    }
     p.n_rblk = static_cast<int32_t>((M + p.RB - 1) / p.RB);
 
     const int pages_max = (st->max_len + p.P - 1) / p.P;
@@ -170,7 +184,11 @@ int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (plan.umma) {
+    if (plan.kernel == Kernel::kPm) {
+        e = launch_attn_pm(p, plan.grid, s);
+        if (e == cudaSuccess)
+            e = p.D == 128 ? launch_attn_merge<128>(p, s) : launch_attn_merge<512>(p, s);
+    } else if (plan.kernel == Kernel::kUmma) {
         e = launch_attn_umma(p, plan.grid, s);
         if (e == cudaSuccess)
             e = launch_attn_merge<128>(p, s);
