@@ -82,6 +82,64 @@ def recorded_traffic(workload):
 def kv_bytes(lens, hkv, d):
     return int(np.sum(np.asarray(lens, dtype=np.int64))) * hkv * d * 2 * 2
 
+PROMPT_METRIC = "chunked prompt attention causal TFLOP/s (fraction of bf16 tensor peak)"
+FALLBACK_TENSOR_TFLOPS = 1400.0
+
+
+def tensor_peak():
+    """Dense bf16 tensor peak: the sustained figure, for kernels timed inside a
+    long run of back-to-back steps."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_TENSOR_TFLOPS, "fallback (sustained)"
+
+
+def throughput(wl, ms, world=1):
+    """The workload's headline unit: causal TFLOP/s for a chunked prompt (tensor
+    bound), K/V GB/s otherwise (HBM bound)."""
+    if wl.w.prompt_len:
+        return world * wl.flops_per_step / (ms * 1e-3) / 1e12, "TFLOP/s"
+    return world * wl.bytes_per_step / (ms * 1e-3) / 1e9, "GB/s"
+
+
+def roofline(wl, attn_ms):
+    """The attention calls (partial + merge kernels) of one step against the bound
+    that limits them."""
+    achieved, unit = throughput(wl, attn_ms)
+    if wl.w.prompt_len:
+        peak, src = tensor_peak()
+        bound = "tensor"
+    else:
+        peak, src = hbm_peak()
+        bound = "hbm"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": recorded_traffic(wl.name),
+            "kernel": "attention calls (partial + merge)", "peak_source": src}
+
+
+def measure_other(name, args, barrier, dist, world, local):
+    import torch
+    wl = Workload(name, f"cuda:{local}")
+    total, attn = time_steps(wl, args.steps, args.warmup, barrier)
+    wl.check_flags()
+    step = total / args.steps
+    if dist is not None:
+        t = torch.tensor([step, attn], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step, attn = t.tolist()
+    value, unit = throughput(wl, step, world)
+    out = {"workload": name, "value": value, "unit": unit, "ms_per_step": step, "attn_ms": attn,
+           "roofline": roofline(wl, attn),
+           "rows_per_s": world * wl.rows_per_step / (step * 1e-3),
+           "gpu_launches": 3 * len(wl.parts()) * args.steps, "config": workload_config(name)}
+    if 1 < wl.w.rows <= 8:
+        out["verify_tokens_per_s"] = out["rows_per_s"]
+    del wl
+    return out
+
 
 # --------------------------------------------------------------------------
 # clocks during the timed region
@@ -148,6 +206,10 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # the workload on the device
 class Workload:
+    """One workload resident on the device.  A step is ``parts()``: (row write,
+    attention call) pairs -- one pair for decode and verify, one per chunk for
+    a chunked prompt (the chunk's rows written, then attended causally)."""
+
     def __init__(self, name, device):
         import torch
         import synth
@@ -156,50 +218,87 @@ class Workload:
         w = synth.WORKLOADS[name]
         self.w = w
         self.name = name
-        self.lens_np = synth.stream_lens(w)
+        W = w.rows
+        if w.prompt_len:
+            assert w.prompt_len % W == 0
+            self.lens_np = np.array([w.prompt_len], dtype=np.int32)
+        else:
+            self.lens_np = synth.stream_lens(w)
         table, n_pages, _ = synth.page_table(w, self.lens_np)
         self.n_pages = n_pages
-        S, W = len(self.lens_np), w.rows
+        S = len(self.lens_np)
         shape = (n_pages, w.n_kv_heads, w.page_size, w.head_dim)
         self.k_pool = torch.full(shape, float("nan"), dtype=torch.bfloat16, device=device)
         self.v_pool = torch.full(shape, float("nan"), dtype=torch.bfloat16, device=device)
         self.table = torch.from_numpy(table).to(device)
         self.lens = torch.from_numpy(self.lens_np).to(device)
         self.max_len = int(self.lens_np.max())
-        new_k, new_v = [], []
-        for s in range(S):
-            n = int(self.lens_np[s])
-            k, v = synth.kv_rows_torch(w, s, n, device)
-            tf.tf_kv_put_rows(self.k_pool, self.v_pool, self.table[s:s + 1], self.lens[s:s + 1],
-                              k[None], v[None], max_len=n)
-            new_k.append(k[n - W:])
-            new_v.append(v[n - W:])
-            del k, v
-        self.k_new = torch.stack(new_k).contiguous()          # [S][W][Hkv][d]
-        self.v_new = torch.stack(new_v).contiguous()
-        self.q = synth.q_rows_torch(w, S, W, device=device)     # [S][W][Hq][d]
+        d, Hq, Hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
+        if w.prompt_len:
+            L = w.prompt_len
+            k, v = synth.kv_rows_torch(w, 0, L, device)
+            self.k_new, self.v_new = k[None].contiguous(), v[None].contiguous()   # [1][L][Hkv][d]
+            self.q = synth.q_rows_torch(w, 1, L, device=device)                  # [1][L][Hq][d]
+            self.chunk_lens = [torch.tensor([W * (c + 1)], dtype=torch.int32, device=device)
+                               for c in range(L // W)]
+            self.bytes_per_step = sum(kv_bytes([W * (c + 1)], Hkv, d) for c in range(L // W))
+            self.flops_per_step = 4 * d * Hq * L * (L + 1) // 2       # causal pairs only
+            self.rows_per_step = L
+        else:
+            new_k, new_v = [], []
+            for s in range(S):
+                n = int(self.lens_np[s])
+                k, v = synth.kv_rows_torch(w, s, n, device)
+                tf.tf_kv_put_rows(self.k_pool, self.v_pool, self.table[s:s + 1], self.lens[s:s + 1],
+                                  k[None], v[None], max_len=n)
+                new_k.append(k[n - W:])
+                new_v.append(v[n - W:])
+                del k, v
+            self.k_new = torch.stack(new_k).contiguous()          # [S][W][Hkv][d]
+            self.v_new = torch.stack(new_v).contiguous()
+            self.q = synth.q_rows_torch(w, S, W, device=device)     # [S][W][Hq][d]
+            self.chunk_lens = None
+            self.bytes_per_step = kv_bytes(self.lens_np, Hkv, d)
+            self.flops_per_step = 4 * d * Hq * sum(
+                int(n) - W + r + 1 for n in self.lens_np for r in range(W))
+            self.rows_per_step = S * W
         self.out = torch.empty(self.q.shape, dtype=torch.float32, device=device)
+        self.bytes_in_l2 = kv_bytes(self.lens_np, Hkv, d) < L2_BYTES
         nbytes = tf.tf_paged_attn_workspace_bytes(self.k_pool, self.v_pool, self.table, self.lens,
-                                                  w.n_q_heads, W, self.max_len)
+                                                  Hq, W, self.max_len)
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         self.attn_fn = (tf.tf_paged_attn_decode if W == 1 else
                         tf.tf_paged_attn_verify if W <= 8 else tf.tf_paged_attn_prompt)
-        self.bytes_per_step = kv_bytes(self.lens_np, w.n_kv_heads, w.head_dim)
-        self.rows_per_step = S * W
         torch.cuda.synchronize()
 
-    def put(self, k_new=None, v_new=None):
-        self.tf.tf_kv_put_rows(self.k_pool, self.v_pool, self.table, self.lens,
-                               self.k_new if k_new is None else k_new,
-                               self.v_new if v_new is None else v_new, max_len=self.max_len)
-
-    def attend(self, q=None):
-        self.attn_fn(self.k_pool, self.v_pool, self.table, self.lens,
-                     self.q if q is None else q, self.w.scale, self.out, self.ws, self.max_len)
+    def parts(self, k_new=None, v_new=None, q=None):
+        """The step's (row write, attention) pairs, optionally on other input buffers."""
+        k_new = self.k_new if k_new is None else k_new
+        v_new = self.v_new if v_new is None else v_new
+        q = self.q if q is None else q
+        tf, w = self.tf, self.w
+        if self.chunk_lens is None:
+            return [(lambda: tf.tf_kv_put_rows(self.k_pool, self.v_pool, self.table, self.lens,
+                                               k_new, v_new, max_len=self.max_len),
+                     lambda: self.attn_fn(self.k_pool, self.v_pool, self.table, self.lens, q,
+                                          w.scale, self.out, self.ws, self.max_len))]
+        W = w.rows
+        out = []
+        for c, lens_c in enumerate(self.chunk_lens):
+            sl = slice(c * W, (c + 1) * W)
+            out.append((
+                lambda sl=sl, lens_c=lens_c: tf.tf_kv_put_rows(
+                    self.k_pool, self.v_pool, self.table, lens_c, k_new[:, sl], v_new[:, sl],
+                    max_len=self.max_len),
+                lambda sl=sl, lens_c=lens_c: self.attn_fn(
+                    self.k_pool, self.v_pool, self.table, lens_c, q[:, sl], w.scale,
+                    self.out[:, sl], self.ws, self.max_len)))
+        return out
 
     def step(self):
-        self.put()
-        self.attend()
+        for put, att in self.parts():
+            put()
+            att()
 
     def check_flags(self):
         torch = self.torch
@@ -210,8 +309,19 @@ class Workload:
             raise RuntimeError(f"device status word set: {flags:#x} (wait sites {site:#x})")
 
 
+L2_BYTES = 126 * 2**20
+
+
 def time_steps(wl, steps, warmup, barrier, sampler=None):
+    """Device time of ``steps`` steps, and the mean per step of the attention
+    calls alone (CUDA events around each call, on the launching stream).  A
+    workload whose K/V fits in L2 gets L2 flushed (a 256 MB write) between
+    steps, outside the per-step events, and its step time is the sum of those."""
     torch = wl.torch
+    parts = wl.parts()
+    flush = None
+    if wl.bytes_in_l2:
+        flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=wl.k_pool.device)
     for _ in range(warmup):
         wl.step()
     torch.cuda.synchronize()
@@ -219,23 +329,32 @@ def time_steps(wl, steps, warmup, barrier, sampler=None):
     stream = torch.cuda.current_stream()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(steps)]
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [[(mk(), mk()) for _ in parts] for _ in range(steps)]
+    sev = [(mk(), mk()) for _ in range(steps)]
     if sampler:
         sampler.mark()
     start.record(stream)
     for i in range(steps):
-        wl.put()
-        ev[i][0].record(stream)
-        wl.attend()
-        ev[i][1].record(stream)
+        if flush is not None:
+            flush.fill_(i & 255)
+        sev[i][0].record(stream)
+        for (put, att), (a, b) in zip(parts, ev[i]):
+            put()
+            a.record(stream)
+            att()
+            b.record(stream)
+        sev[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     if sampler:
         sampler.mark()
     barrier()
-    total_ms = start.elapsed_time(end)
-    attn_ms = [a.elapsed_time(b) for a, b in ev]
+    if flush is not None:
+        total_ms = sum(a.elapsed_time(b) for a, b in sev)
+    else:
+        total_ms = start.elapsed_time(end)
+    attn_ms = [sum(a.elapsed_time(b) for a, b in step) for step in ev]
     return total_ms, statistics.mean(attn_ms)
 
 
@@ -247,13 +366,15 @@ def time_e2e(wl, steps, warmup, barrier):
     v_h = wl.v_new.cpu().pin_memory()
     out_h = torch.empty(wl.out.shape, dtype=torch.float32).pin_memory()
     q_d, k_d, v_d = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
+    parts = wl.parts(k_d, v_d, q_d)
 
     def one():
         q_d.copy_(q_h, non_blocking=True)
         k_d.copy_(k_h, non_blocking=True)
         v_d.copy_(v_h, non_blocking=True)
-        wl.put(k_d, v_d)
-        wl.attend(q_d)
+        for put, att in parts:
+            put()
+            att()
         out_h.copy_(wl.out, non_blocking=True)
 
     for _ in range(warmup):
@@ -311,20 +432,30 @@ def oracle_sample(wl_name, n_units, threads, device_kv=None):
     oracle.attend(q, k_lin, v_lin, lens[:1], w.rows, w.group, w.scale, units=units,
                   threads=threads)
     dt = time.perf_counter() - t0
-    per_unit = w.head_dim * 2 * 2 / w.group          # one query head's share of a K/V row
-    nbytes = sum((n0 - w.rows + int(r) + 1) * per_unit for _, r, _ in units)
+    visible = [n0 - w.rows + int(r) + 1 for _, r, _ in units]
+    if w.prompt_len:
+        # causal flops of the sampled rows (q.k and p.v: 4 d per visible position)
+        work = sum(4 * w.head_dim * n for n in visible) / 1e12
+    else:
+        per_unit = w.head_dim * 2 * 2 / w.group      # one query head's share of a K/V row
+        work = sum(n * per_unit for n in visible) / 1e9
     desc = (f"{len(units)} (stream, row, query head) output rows of stream 0 at {n0} positions "
             f"(the stream's {len(base)} rows, repeated), fp64, {threads} threads")
-    return dt, nbytes, desc
+    return dt, work, desc
 
 
 def cpu_baseline(wl_name, device_kv, budget_s=12.0):
     threads = os.cpu_count() or 1
     dt1, _, _ = oracle_sample(wl_name, threads, threads, device_kv)
     n = int(max(threads, budget_s / max(dt1, 1e-3) * threads))
-    dt, nbytes, desc = oracle_sample(wl_name, n, threads, device_kv)
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+    dt, work, desc = oracle_sample(wl_name, n, threads, device_kv)
+    return {"value": work / dt, "unit": oracle_unit(wl_name), "cores": threads, "kind": "oracle",
             "sample": desc, "seconds": round(dt, 3)}
+
+
+def oracle_unit(wl_name):
+    import synth
+    return "TFLOP/s" if synth.WORKLOADS[wl_name].prompt_len else "GB/s"
 
 
 def run_reference(args):
@@ -340,20 +471,22 @@ def run_reference(args):
     n_units = int(max(1, per_step / max(dt1, 1e-3) * threads))
     for _ in range(args.warmup):
         oracle_sample(args.workload, n_units, threads)
-    secs, nbytes = 0.0, 0.0
+    secs, work = 0.0, 0.0
     desc = ""
     for _ in range(args.steps):
-        dt, nb, desc = oracle_sample(args.workload, n_units, threads)
+        dt, wk, desc = oracle_sample(args.workload, n_units, threads)
         secs += dt
-        nbytes += nb
-    value = nbytes / secs / 1e9
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 0,
+        work += wk
+    value = work / secs
+    unit = oracle_unit(args.workload)
+    line = {"impl": "reference", "metric": METRIC if unit == "GB/s" else PROMPT_METRIC,
+            "value": value, "unit": unit, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(args.workload),
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                              "sample": desc},
-            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -363,10 +496,15 @@ def workload_config(name):
     import synth
     w = synth.WORKLOADS[name]
     lens = synth.stream_lens(w)
-    return {"workload": name, "streams": len(lens), "context": int(lens.max()),
-            "kv_heads": w.n_kv_heads, "q_heads": w.n_q_heads, "head_dim": w.head_dim,
-            "page_size": w.page_size, "rows": w.rows, "parallelism": "replicas",
-            "l2": f"inputs {kv_bytes(lens, w.n_kv_heads, w.head_dim) / 1e9:.2f} GB > 126 MB L2"}
+    cfg = {"workload": name, "streams": len(lens), "context": int(lens.max()),
+           "kv_heads": w.n_kv_heads, "q_heads": w.n_q_heads, "head_dim": w.head_dim,
+           "page_size": w.page_size, "rows": w.rows, "parallelism": "replicas",
+           "l2": f"inputs {kv_bytes(lens, w.n_kv_heads, w.head_dim) / 1e9:.2f} GB > 126 MB L2"}
+    if w.prompt_len:
+        cfg["chunks"] = w.prompt_len // w.rows
+        cfg["l2"] = (f"K/V {kv_bytes(lens, w.n_kv_heads, w.head_dim) / 1e6:.1f} MB < 126 MB L2: "
+                     "L2 flushed (256 MB write) between timed steps, outside the step's events")
+    return cfg
 
 
 # --------------------------------------------------------------------------
@@ -409,30 +547,7 @@ def main():
     wl.check_flags()
     e2e_ms, h2d, d2h = time_e2e(wl, args.steps, args.warmup, barrier)
     wl.check_flags()
-    bytes_per_step, rows_per_step = wl.bytes_per_step, wl.rows_per_step
-
-    # the metric's second half: verify tokens/s on the draft-verify workload
-    secondary = None
-    if args.workload == "decode_12x40k" and not args.no_verify:
-        del wl
-        torch.cuda.empty_cache()
-        vw = Workload("verify_4x131k", f"cuda:{local}")
-        v_total, v_attn = time_steps(vw, args.steps, args.warmup, barrier)
-        vw.check_flags()
-        v_step = v_total / args.steps
-        if dist is not None:
-            t = torch.tensor([v_step, v_attn], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            v_step, v_attn = t.tolist()
-        v_ach = vw.bytes_per_step / (v_attn * 1e-3) / 1e9
-        peak_v, _ = hbm_peak()
-        secondary = {"workload": "verify_4x131k", "verify_tokens_per_s": world * vw.rows_per_step / (v_step * 1e-3),
-                     "kv_gbs": world * vw.bytes_per_step / (v_step * 1e-3) / 1e9, "ms_per_step": v_step,
-                     "attn_ms": v_attn, "roofline_frac": v_ach / peak_v,
-                     "traffic": recorded_traffic("verify_4x131k"),
-                     "gpu_launches": 3 * args.steps, "config": workload_config("verify_4x131k")}
-        del vw
-        torch.cuda.empty_cache()
+    n_parts = len(wl.parts())
 
     ms_step = total_ms / args.steps
     e2e_step = e2e_ms / args.steps
@@ -440,27 +555,33 @@ def main():
         t = torch.tensor([ms_step, e2e_step, attn_ms], device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step, e2e_step, attn_ms = t.tolist()
-    value = world * bytes_per_step / (ms_step * 1e-3) / 1e9
-    e2e_value = world * bytes_per_step / (e2e_step * 1e-3) / 1e9
-    peak, src = hbm_peak()
-    achieved = bytes_per_step / (attn_ms * 1e-3) / 1e9
+    value, unit = throughput(wl, ms_step, world)
+    e2e_value, _ = throughput(wl, e2e_step, world)
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if not wl.w.prompt_len else PROMPT_METRIC,
+        "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(args.workload),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(args.workload),
-                     "kernel": "attention call (partial + merge)", "peak_source": src},
-        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+        "roofline": roofline(wl, attn_ms),
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 3 * n_parts * args.steps,
         "clocks": sampler.summary(),
-        "rows_per_s": world * rows_per_step / (ms_step * 1e-3),
+        "rows_per_s": world * wl.rows_per_step / (ms_step * 1e-3),
         "attn_ms": attn_ms,
     }
-    if secondary is not None:
-        line["verify"] = secondary
+    del wl
+    torch.cuda.empty_cache()
+
+    # the metric's second half (verify tokens/s) and the other workloads, each
+    # timed the same way on its own
+    if args.workload == "decode_12x40k" and not args.no_verify:
+        for name, key in (("verify_4x131k", "verify"), ("hd512_verify", "hd512"),
+                          ("prompt_9216", "prompt")):
+            line[key] = measure_other(name, args, barrier, dist, world, local)
+            torch.cuda.empty_cache()
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth
         w0 = synth.WORKLOADS[args.workload]

@@ -170,3 +170,48 @@ def test_parity_growing_scores(d, G, W):
                         threads=8)
     assert torch.isfinite(out).all()
     assert max_abs(out, ref) <= TOL
+
+
+# --- the stream-K split: every CTA gets an equal run of 128-position tiles
+# across the call's (stream, KV head, row block) units; these cases put the
+# split's corners under the oracle.
+
+@pytest.mark.parametrize("d,G,W", [(128, 4, 1), (128, 8, 8), (512, 8, 4), (128, 4, 64)])
+def test_split_fewer_tiles_than_ctas(d, G, W):
+    """A handful of one-tile units: most CTAs get an empty range."""
+    w = small_workload(d, G, 512, W, seed=9000 + d + G + W)
+    run_parity(w, [W + 5, 100, 127, 128], W)
+
+
+@pytest.mark.parametrize("d,G,W", [(128, 4, 1), (128, 8, 8), (512, 8, 4), (128, 4, 128)])
+def test_split_one_long_stream(d, G, W):
+    """One stream and one KV head: its units are split over every CTA, and the
+    merge combines about one segment per CTA."""
+    w = synth.Workload("one", 0, 1, G, d, 512, W, seed=9100 + d + G + W)
+    run_parity(w, [40000 if d == 128 else 12000], W)
+
+
+def test_split_many_short_streams():
+    """Many short streams: a CTA's range runs over many whole units."""
+    rng = np.random.default_rng(9200)
+    lens = [int(x) for x in rng.integers(8, 700, size=60)] + [5000, 8, 1]
+    w = small_workload(128, 8, 512, 1, Hkv=2, seed=9201)
+    run_parity(w, lens, 1)
+
+
+def test_split_skips_out_of_range_stream():
+    """A stream longer than max_len in the middle of the call: its rows are NaN
+    and flagged, and the split over the other streams is unaffected."""
+    import verify_paged_gqa_b200 as tf
+    w = small_workload(128, 8, 512, 4, seed=9300)
+    case = synth.make_case(w, lens=[3000, 2500, 4000], rows=4)
+    dc = DeviceCase(case)
+    ws = dc.workspace(4)
+    lens = torch.tensor([3000, 2500, 4000], dtype=torch.int32, device="cuda")
+    out = dc.attend(lens=lens, max_len=3500, ws=ws)
+    assert tf.tf_workspace_status(ws) & tf.TF_DEV_BAD_LEN
+    assert torch.isnan(out[2]).all()
+    keep = [0, 1]
+    ref = oracle.attend(case.q[keep], [case.k_lin[i] for i in keep], [case.v_lin[i] for i in keep],
+                        case.lens[keep], 4, w.group, w.scale, threads=8)
+    assert max_abs(out[keep], ref) <= TOL

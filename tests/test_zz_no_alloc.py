@@ -51,14 +51,14 @@ def test_noalloc_decode_matches_workspace_decode_twice(d, G, lens):
 
 def test_noalloc_refuses_a_plan_beyond_its_scratch():
     import verify_paged_gqa_b200 as tf
-    # 64 streams x 8 KV heads at 131,072 positions needs far more than 8 MiB of partials
-    w = synth.Workload("noalloc_big", 0, 8, 4, 128, 512, 1, seed=8100)
-    S, L = 64, 131072
-    pages = S * (L // 512)
-    k_pool = torch.empty((1, 8, 512, 128), dtype=torch.bfloat16, device="cuda")
-    table = torch.zeros((S, L // 512), dtype=torch.int32, device="cuda")
+    # 64 query heads on one KV head at head dim 512: two row blocks of 32 rows,
+    # and two partial slots of 32 x 514 floats per CTA -- more than 8 MiB
+    w = synth.Workload("noalloc_big", 0, 1, 64, 512, 512, 1, seed=8100)
+    S, L = 4, 4096
+    k_pool = torch.empty((S * L // 512, 1, 512, 512), dtype=torch.bfloat16, device="cuda")
+    table = torch.arange(S * L // 512, dtype=torch.int32, device="cuda").view(S, L // 512)
     lens = torch.full((S,), L, dtype=torch.int32, device="cuda")
-    q = torch.zeros((S, 1, 32, 128), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((S, 1, 64, 512), dtype=torch.bfloat16, device="cuda")
     out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
 
     class _DC:
@@ -66,6 +66,6 @@ def test_noalloc_refuses_a_plan_beyond_its_scratch():
     dc = _DC()
     dc.k_pool = dc.v_pool = k_pool
     dc.table, dc.lens, dc.max_len, dc.w = table, lens, L, w
-    need = tf.tf_paged_attn_workspace_bytes(k_pool, k_pool, table, lens, 32, 1, L)
-    assert need > (8 << 20) and pages > 0
+    need = tf.tf_paged_attn_workspace_bytes(k_pool, k_pool, table, lens, 64, 1, L)
+    assert need > (8 << 20)
     assert _noalloc(tf, dc, q, out) == tf.TF_ENOSPACE

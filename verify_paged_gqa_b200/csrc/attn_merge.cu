@@ -8,22 +8,28 @@
 //     m* = max_c m_c,   w_c = 2^(m_c - m*),
 //     out = (sum_c w_c O_c) / (sum_c w_c l_c)
 // The maximum and the sum of l are warp-shuffle reductions; the O sum runs
-// in chunk order, so the result is the same on every run.
+// in segment (position) order, so the result is the same on every run.
 //
-// One block per (stream, KV head, row block, group of up to 8 rows); one
-// warp per row.  Streams whose length is out of range get NaN rows (and the
-// status bit).
+// The segments of a unit split across CTAs are found from the tile split
+// (plan.cuh): the CTAs whose ranges meet the unit's tiles [U0, U1), in
+// order.  One block per (stream, KV head, row block, group of up to 8 rows);
+// one warp per row.  The weighted sum loads several segments' rows before
+// using them, so the loads of a round overlap.  Streams whose length is out
+// of range get NaN rows (and the status bit).
 #include "launch.cuh"
 #include "plan.cuh"
 
 namespace tfp {
 
-constexpr int kMergeRows = 8;  // rows (warps) per merge block
+constexpr int kMergeRows = 8;    // rows (warps) per merge block
 
 template <int D>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__ AttnParams p)
 {
-    constexpr int DL = D / 32;
+    constexpr int DL = D / 32;            // output floats per lane
+    constexpr int NV = DL / 4;            // float4 per lane and segment
+    constexpr int UK = D == 128 ? 8 : 4;  // segments loaded per round
+    __shared__ int slots[kMaxCtas];       // partial slot of each segment, -1: none
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int nwarps = blockDim.x / 32;
@@ -55,24 +61,45 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
         }
         return;
     }
-    const int nc = block_chunks(p, len, b);
-    if (nc <= 1)
-        return;  // the partial kernel wrote the output itself
-    const size_t slot_floats = (size_t)p.RB * (D + 2);
-    const float *base = p.part + part_slot(p, s, kh, b, 0) * slot_floats;
+    // the unit's tiles [U0, U1) and the CTAs that met them
+    const long long tot = *p.total_tiles;
+    long long U0 = p.first_tile[s] + kh * head_tiles(p, len);
+    for (int bb = 0; bb < b; ++bb)
+        U0 += unit_tiles(p, len, bb);
+    const long long U1 = U0 + unit_tiles(p, len, b);
+    const int c_lo = cta_of(U0, tot, p.n_cta);
+    const int c_hi = cta_of(U1 - 1, tot, p.n_cta);
+    if (c_lo == c_hi)
+        return;  // one segment covered the unit and wrote the rows itself
+    const int nseg = min(c_hi - c_lo + 1, kMaxCtas);
+    for (int k = threadIdx.x; k < nseg; k += blockDim.x) {
+        const int c = c_lo + k;
+        const long long a0 = range_start(tot, c, p.n_cta);
+        const long long a1 = range_start(tot, c + 1, p.n_cta);
+        // the first CTA's segment is its last unless its range starts at U0
+        slots[k] = a0 == a1 ? -1 : (k == 0 && a0 < U0) ? 2 * c + 1 : 2 * c;
+    }
+    __syncthreads();
+    const size_t slot_floats = (size_t)p.SR * (D + 2);
 
     for (int m = m0 + warp; m < m1; m += nwarps) {
         const int r = m - mb;
         float mx = NEG_INF;
-        for (int c = lane; c < nc; c += 32)
-            mx = fmaxf(mx, base[c * slot_floats + (size_t)p.RB * D + r]);
+        for (int k = lane; k < nseg; k += 32) {
+            const int sl = slots[k];
+            if (sl >= 0)
+                mx = fmaxf(mx, p.part[sl * slot_floats + (size_t)p.SR * D + r]);
+        }
 #pragma unroll
         for (int k = 16; k >= 1; k >>= 1)
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, k));
         float l = 0.f;
-        for (int c = lane; c < nc; c += 32) {
-            const float mc = base[c * slot_floats + (size_t)p.RB * D + r];
-            const float lc = base[c * slot_floats + (size_t)p.RB * D + p.RB + r];
+        for (int k = lane; k < nseg; k += 32) {
+            const int sl = slots[k];
+            if (sl < 0)
+                continue;
+            const float mc = p.part[sl * slot_floats + (size_t)p.SR * D + r];
+            const float lc = p.part[sl * slot_floats + (size_t)p.SR * D + p.SR + r];
             l += (mc == NEG_INF) ? 0.f : lc * fast_exp2(mc - mx);
         }
 #pragma unroll
@@ -83,18 +110,35 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
 #pragma unroll
         for (int e = 0; e < DL; ++e)
             acc[e] = 0.f;
-        for (int c = 0; c < nc; ++c) {
-            const float *sl = base + c * slot_floats;
-            const float mc = sl[(size_t)p.RB * D + r];
-            const float w = (mc == NEG_INF) ? 0.f : fast_exp2(mc - mx);
-            const float *orow = sl + (size_t)r * D;
+        for (int k0 = 0; k0 < nseg; k0 += UK) {
+            float w[UK];
+            float4 v[UK][NV];
 #pragma unroll
-            for (int q = 0; q < DL / 4; ++q) {
-                const float4 v = *reinterpret_cast<const float4 *>(orow + q * 128 + lane * 4);
-                acc[q * 4 + 0] = fmaf(w, v.x, acc[q * 4 + 0]);
-                acc[q * 4 + 1] = fmaf(w, v.y, acc[q * 4 + 1]);
-                acc[q * 4 + 2] = fmaf(w, v.z, acc[q * 4 + 2]);
-                acc[q * 4 + 3] = fmaf(w, v.w, acc[q * 4 + 3]);
+            for (int kk = 0; kk < UK; ++kk) {
+                const int sl = k0 + kk < nseg ? slots[k0 + kk] : -1;
+                w[kk] = 0.f;
+#pragma unroll
+                for (int q = 0; q < NV; ++q)
+                    v[kk][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (sl >= 0) {
+                    const float *base = p.part + sl * slot_floats;
+                    const float mc = base[(size_t)p.SR * D + r];
+                    w[kk] = (mc == NEG_INF) ? 0.f : fast_exp2(mc - mx);
+#pragma unroll
+                    for (int q = 0; q < NV; ++q)
+                        v[kk][q] = *reinterpret_cast<const float4 *>(base + (size_t)r * D + q * 128 +
+                                                                     lane * 4);
+                }
+            }
+#pragma unroll
+            for (int kk = 0; kk < UK; ++kk) {
+#pragma unroll
+                for (int q = 0; q < NV; ++q) {
+                    acc[q * 4 + 0] = fmaf(w[kk], v[kk][q].x, acc[q * 4 + 0]);
+                    acc[q * 4 + 1] = fmaf(w[kk], v[kk][q].y, acc[q * 4 + 1]);
+                    acc[q * 4 + 2] = fmaf(w[kk], v[kk][q].z, acc[q * 4 + 2]);
+                    acc[q * 4 + 3] = fmaf(w[kk], v[kk][q].w, acc[q * 4 + 3]);
+                }
             }
         }
         const float inv = 1.f / l;
@@ -102,7 +146,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
         const int h = kh * p.G + (m - wr * p.G);
         float *orow = p.out + (((size_t)s * p.W + wr) * p.Hq + h) * D;
 #pragma unroll
-        for (int q = 0; q < DL / 4; ++q)
+        for (int q = 0; q < NV; ++q)
             *reinterpret_cast<float4 *>(orow + q * 128 + lane * 4) =
                 make_float4(acc[q * 4 + 0] * inv, acc[q * 4 + 1] * inv, acc[q * 4 + 2] * inv,
                             acc[q * 4 + 3] * inv);

@@ -31,12 +31,12 @@
 //              so the softmax of one tile overlaps the MMAs of the next.
 //              Owns the tensor-memory allocation.
 //   warps 2-5  softmax, one key position per thread: write the block's query
-//              rows into the Q tile at each item's start; per tile, read the
+//              rows into the Q tile at each segment's start; per tile, read the
 //              position's scores for all rows, check them against each row's
 //              reference max (a block-wide vote; the reference moves only
 //              when some row's max grows by more than 2^8, and then O^T is
 //              rescaled), write P^T, and keep per-thread row sums.  At the
-//              item's end the sums are reduced across the block and the rows
+//              segment's end the sums are reduced across the block and the rows
 //              are normalised and stored, or left as partials for the merge.
 #include "launch.cuh"
 #include "plan.cuh"
@@ -63,8 +63,12 @@ struct PmCfg {
     static constexpr uint32_t kCols = 2 * NR + DB * 2 * NR;
     static constexpr uint32_t kTmemCols =
         kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
-    static constexpr uint32_t kSmall = 48 * NR + 512;  // per-row arrays and barriers
-    static constexpr int kFit = (int)((kSmemCap - 1024 - kQBytes - 2 * kPBytes - kSmall) / kUnit);
+    static constexpr uint32_t kSmall = 48 * NR + 512;  // per-row arrays, range, barriers
+    // P^T buffers: with one, the softmax of tile t + 1 stores P only after
+    // PV(t) completed, and the shared memory goes to the K/V ring instead
+    static constexpr int kPBufs = 2;
+    static constexpr int kFit =
+        (int)((kSmemCap - 1024 - kQBytes - kPBufs * kPBytes - kSmall) / kUnit);
     static constexpr int NU = kFit > 6 ? 6 : kFit;     // ring units
     static_assert(kCols <= 512, "tensor memory");
     static_assert(NU >= 2, "ring");
@@ -78,17 +82,18 @@ struct PmSmem {
     using C = PmCfg<D, NR>;
     alignas(1024) uint8_t ring[C::NU][kUnit];
     alignas(1024) uint8_t q[C::kQBytes];
-    alignas(1024) uint8_t pt[2][C::kPBytes];
+    alignas(1024) uint8_t pt[C::kPBufs][C::kPBytes];
     alignas(16) float mref[NR];   // row reference max, log2 units; -inf while the row saw nothing
     alignas(16) float negm[NR];   // -mref, or +inf while mref is -inf (forces a new reference)
     alignas(16) float alpha[NR];  // factor of the last reference change
     alignas(16) float lsum[NR];   // row sums (inverted for a finished row block)
     alignas(16) float red[4][NR];
-    long long rowoff[2][NR];      // output offset of row r (by item parity); -1 past M
+    long long rowoff[2][NR];      // output offset of row r (by segment parity); -1 past M
+    CtaRange range;               // this CTA's tiles
     uint64_t full[C::NU];
     uint64_t empty[C::NU];
-    uint64_t q_full;      // the softmax warps wrote the item's Q tile
-    uint64_t q_free;      // the item's last QK MMA is done with the Q tile
+    uint64_t q_full;      // the softmax warps wrote the segment's Q tile
+    uint64_t q_free;      // the segment's last QK MMA is done with the Q tile
     uint64_t s_full[2];   // S^T(t) is in tensor memory
     uint64_t p_full[2];   // the softmax warps wrote P^T(t)
     uint64_t o_done[2];   // the PV reading P^T buffer b (and every MMA before it) completed
@@ -211,7 +216,7 @@ __device__ __forceinline__ bool pm_put_tile(const AttnParams &p, PmSmem<D, NR> &
     return true;
 }
 
-// Unit order per item (the issuer consumes in the same order):
+// Unit order per segment (the issuer consumes in the same order):
 // K(0), then for each tile t: K(t + 1) if any, V(t).
 template <int D, int NR>
 __device__ __forceinline__ void pm_producer(const PmArgs &a, PmSmem<D, NR> &sm)
@@ -219,12 +224,12 @@ __device__ __forceinline__ void pm_producer(const PmArgs &a, PmSmem<D, NR> &sm)
     using C = PmCfg<D, NR>;
     const AttnParams &p = a.p;
     const uint64_t pol = l2_evict_first_policy();
-    ItemCursor cur;
-    cur.init();
+    SegCursor cur;
+    cur.init(p, sm.range);
     WorkItem it;
     uint32_t U = 0;
     bool ok = true;
-    for (int64_t i = blockIdx.x; ok && cur.seek(p, i, it); i += gridDim.x) {
+    while (ok && cur.next(p, it)) {
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
         int pg0 = __ldg(trow + it.key0 / p.P);
@@ -291,12 +296,12 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
     const uint32_t q0 = smem_addr(sm.q);
     const uint32_t pt0 = smem_addr(sm.pt[0]);
 
-    ItemCursor cur;
-    cur.init();
+    SegCursor cur;
+    cur.init(p, sm.range);
     WorkItem it;
     uint32_t U = 0, T0 = 0, j = 0;
     bool ok = true;
-    for (int64_t i = blockIdx.x; ok && cur.seek(p, i, it); i += gridDim.x, ++j) {
+    for (; ok && cur.next(p, it); ++j) {
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         ok = pwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
         tc_fence_after();
@@ -320,7 +325,7 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
             tc_fence_after();
             if (!ok)
                 break;
-            const uint32_t pb = pt0 + (T & 1u) * C::kPBytes;
+            const uint32_t pb = pt0 + (T % C::kPBufs) * C::kPBytes;
 #pragma unroll 1
             for (int vb = 0; vb < C::DB; ++vb) {
                 const int st = (int)(U % C::NU);
@@ -371,12 +376,12 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
     const int sw = tid & 7;
     const int R0 = 32 * h;               // first row of this thread
 
-    ItemCursor cur;
-    cur.init();
-    WorkItem it;
+    SegCursor cur;
+    cur.init(p, sm.range);
+    WorkItem it, nx;
     uint32_t j = 0, u0 = 0;
     bool ok = true;
-    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
+    for (; cur.next(p, it); ++j) {
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         // --- the block's query rows into the Q tile; output offsets ---------
         {
@@ -392,15 +397,14 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                 }
                 sm.rowoff[j & 1u][st] = off;
             }
-            // (already complete in practice: the previous item's last PV,
+            // (already complete in practice: the previous segment's last PV,
             // waited for below, was issued after its last QK)
             ok = pwait(sm, &sm.q_free, (j & 1u) ^ 1u, p.flags, kWaitQEmpty) && ok;
+            {
+                uint4 qv[kPer];
 #pragma unroll
-            for (int c0 = 0; c0 < kPer; c0 += 4) {
-                uint4 qv[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int f = st + NT * (c0 + c);
+                for (int c = 0; c < kPer; ++c) {
+                    const int f = st + NT * c;
                     const int r = f / (D / 8), k = f % (D / 8);
                     const int m = it.b * NR + r;
                     qv[c] = make_uint4(0, 0, 0, 0);
@@ -413,11 +417,27 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                     }
                 }
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int f = st + NT * (c0 + c);
+                for (int c = 0; c < kPer; ++c) {
+                    const int f = st + NT * c;
                     const int r = f / (D / 8), k = f % (D / 8);
                     *reinterpret_cast<uint4 *>(sm.q + (k >> 3) * (NR * 128) + sw128_off(r, k & 7)) =
                         qv[c];
+                }
+            }
+            // the next segment's query rows into L2 (128-byte lines)
+            SegCursor ahead = cur;
+            if (ahead.next(p, nx)) {
+                constexpr int kLines = NR * D * 2 / 128;
+                for (int f = st; f < kLines; f += NT) {
+                    const int r = f / (D / 64), k = f % (D / 64);
+                    const int m = nx.b * NR + r;
+                    if (m < p.M) {
+                        const int wr = m / p.G;
+                        const int hq = nx.kh * p.G + (m - wr * p.G);
+                        const __nv_bfloat16 *src =
+                            p.q + (((size_t)nx.s * p.W + wr) * p.Hq + hq) * D + k * 64;
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
+                    }
                 }
             }
             fence_async_smem();
@@ -554,34 +574,36 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                     }
                 }
             }
-            // --- P^T(u): buffer u & 1 is free once PV(u - 2) completed -----
-            if (u >= 2)
-                ok = pwait(sm, &sm.o_done[u & 1u], ((u - 2) >> 1) & 1u, p.flags, kWaitEmpty) && ok;
-            uint8_t *pr = sm.pt[u & 1u] + prow;
+            // --- P^T(u) -----------------------------------------------------
+            uint32_t hw[16], lw[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float p0 = fast_exp2(x[2 * e]);
+                const float p1 = fast_exp2(x[2 * e + 1]);
+                l[2 * e] += p0;
+                l[2 * e + 1] += p1;
+                // P = hi + lo, both bf16 by truncation: |p - hi - lo| < 2^-14 p
+                const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+                hw[e] = __byte_perm(b0, b1, 0x7632);
+                const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
+                const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
+                lw[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+            }
+            // buffer u % kPBufs is free once PV(u - kPBufs) completed
+            if (u >= (uint32_t)C::kPBufs) {
+                const uint32_t v = u - C::kPBufs;
+                ok = pwait(sm, &sm.o_done[v & 1u], (v >> 1) & 1u, p.flags, kWaitEmpty) && ok;
+            }
+            uint8_t *pr = sm.pt[u % C::kPBufs] + prow;
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int r = 8 * g + 2 * e;
-                    const float p0 = fast_exp2(x[r]);
-                    const float p1 = fast_exp2(x[r + 1]);
-                    l[r] += p0;
-                    l[r + 1] += p1;
-                    // P = hi + lo, both bf16 by truncation: |p - hi - lo| < 2^-14 p
-                    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
-                    hw[e] = __byte_perm(b0, b1, 0x7632);
-                    const float r0 = p0 - __uint_as_float(b0 & 0xffff0000u);
-                    const float r1 = p1 - __uint_as_float(b1 & 0xffff0000u);
-                    lw[e] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
-                }
                 // hi of rows R0 + 8g .. + 7 is 16-byte chunk R0 / 8 + g of the
                 // position's row; lo is chunk (NR + R0) / 8 + g
                 const int ch = R0 / 8 + g, cl = (NR + R0) / 8 + g;
                 *reinterpret_cast<uint4 *>(pr + (ch >> 3) * kBox + (((ch & 7) ^ sw) << 4)) =
-                    make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    make_uint4(hw[4 * g], hw[4 * g + 1], hw[4 * g + 2], hw[4 * g + 3]);
                 *reinterpret_cast<uint4 *>(pr + (cl >> 3) * kBox + (((cl & 7) ^ sw) << 4)) =
-                    make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    make_uint4(lw[4 * g], lw[4 * g + 1], lw[4 * g + 2], lw[4 * g + 3]);
             }
             fence_async_smem();
             tc_fence_before();
@@ -590,11 +612,11 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                 mbar_arrive(&sm.p_full[u & 1u]);
         }
 
-        // --- the item's last PV, then the rows' results ------------------------
+        // --- the segment's last PV, then the rows' results ------------------------
         const uint32_t ulast = u0 + n - 1;
         ok = pwait(sm, &sm.o_done[ulast & 1u], (ulast >> 1) & 1u, p.flags, kWaitEmpty) && ok;
         tc_fence_after();
-        const bool fin = it.nc == 1;
+        const bool fin = it.fin;
         xpose_reduce<32, false>(l, lane);
         sm.red[wq][R0 + lane] = l[0];
         named_barrier(1, NT);
@@ -605,7 +627,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
         named_barrier(1, NT);
         const bool write = ok && !sm.abort_flag;
         float *slot = fin ? nullptr
-                          : p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(NR * (D + 2));
+                          : p.part + (size_t)it.slot * (p.SR * (D + 2));
 #pragma unroll 1
         for (int vb = 0; vb < C::DB; ++vb) {
             uint32_t hi[32], lo[32];
@@ -622,15 +644,15 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                         const long long off = sm.rowoff[j & 1u][r];
                         if (off >= 0)
                             p.out[off + d] = o * sm.lsum[r];
-                    } else {
+                    } else if (r < p.SR) {
                         slot[(size_t)r * D + d] = o;
                     }
                 }
             }
         }
-        if (write && !fin && st < NR) {
-            slot[(size_t)NR * D + st] = sm.mref[st];
-            slot[(size_t)NR * D + NR + st] = sm.lsum[st];
+        if (write && !fin && st < p.SR) {
+            slot[(size_t)p.SR * D + st] = sm.mref[st];
+            slot[(size_t)p.SR * D + p.SR + st] = sm.lsum[st];
         }
         tc_fence_before();
         u0 += n;
@@ -663,6 +685,8 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == 0)
+        find_range(a.p, sm.range, lane);
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr(&sm.tmem_base)), "r"(C::kTmemCols)

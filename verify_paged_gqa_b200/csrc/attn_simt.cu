@@ -10,8 +10,8 @@
 // first tile is needed.
 //
 // Layout of one CTA (persistent, one per SM):
-//   last warp     producer (one lane): walks the CTA's work items one item
-//                 ahead; per item it copies the four query rows into a
+//   last warp     producer (one lane): walks the CTA's segments one segment
+//                 ahead; per segment it copies the four query rows into a
 //                 double-buffered shared slot and streams K and V tiles of TK
 //                 positions into a ring of NSTAGE stages with bulk copies
 //                 (TMA engine, no tensor map: a tile of one page and KV head
@@ -19,12 +19,12 @@
 //   other warps   consumers: tile T of the CTA's sequence goes to consumer
 //                 warp T % NCW.  A warp keeps its own online-softmax state
 //                 (running max m, running sum l, unnormalised O) for the four
-//                 rows of the item.  At the end of the item each warp parks
+//                 rows of the segment.  At the end of the segment each warp parks
 //                 its state in shared memory; the last warp to arrive
-//                 combines them and writes the item's result (the normalised
+//                 combines them and writes the segment's result (the normalised
 //                 output when the row block has one chunk, else a partial for
 //                 the merge kernel).  No CTA-wide barrier: the other warps go
-//                 straight on to the next item.
+//                 straight on to the next segment.
 //
 // Inner loop of a consumer warp on one tile (head dim 128, TK = 32):
 //   scores  the warp is 4 groups of 8 lanes; group g takes 8 keys, lane i of
@@ -40,7 +40,7 @@
 //   PV      lane L owns dims 4L..4L+3 of the 4 output rows as fp32 pairs and
 //           updates them with packed fp32 FMAs (two per instruction);
 //           probabilities come from a per-warp shared buffer; only positions
-//           below the item's end are visited, so no unused slot is read.
+//           below the segment's end are visited, so no unused slot is read.
 // Head dim 512 uses TK = 8 and one group of 32 lanes; the same steps.
 #include "launch.cuh"
 #include "plan.cuh"
@@ -77,7 +77,7 @@ struct SimtSmem {
     static constexpr int NCW = SimtCfg<D>::NCW;
     static constexpr int TILE_BYTES = TK * D * 2;
     alignas(128) uint8_t kv[NSTAGE][2][TILE_BYTES];
-    alignas(16) __nv_bfloat16 qbuf[2][kR][D];      // the item's query rows (double buffer)
+    alignas(16) __nv_bfloat16 qbuf[2][kR][D];      // the segment's query rows (double buffer)
     alignas(16) float pbuf[NCW][TK][2 * kR];        // per key: p0,p0,p1,p1,p2,p2,p3,p3
     alignas(16) float wo[NCW][kR][D];               // parked warp states
     float wm[NCW][kR];
@@ -94,7 +94,8 @@ struct SimtSmem {
     uint64_t q_full[2];
     uint64_t q_empty[2];
     uint64_t w_free;       // the parked-state slot is free again (combine done)
-    int w_count;           // warps parked for the current item
+    int w_count;           // warps parked for the current segment
+    CtaRange range;        // this CTA's tiles
     volatile int abort_flag;
 };
 
@@ -173,7 +174,7 @@ __device__ __forceinline__ bool wait_tag(SimtSmem<D> &sm, int stage, uint32_t T,
     return true;
 }
 
-// Copies the four query rows of item `it` into q slot (j & 1).
+// Copies the four query rows of segment `it` into q slot (j & 1).
 template <int D>
 __device__ __forceinline__ bool producer_q(const AttnParams &p, SimtSmem<D> &sm,
                                            const WorkItem &it, uint32_t j, uint64_t pol)
@@ -192,8 +193,8 @@ __device__ __forceinline__ bool producer_q(const AttnParams &p, SimtSmem<D> &sm,
     return true;
 }
 
-// One lane.  Looks one item ahead: the next item's query rows are copied
-// when the current item starts, and every page id is read one page before
+// One lane.  Looks one segment ahead: the next segment's query rows are copied
+// when the current segment starts, and every page id is read one page before
 // its first tile, so no table read sits on the copy path.
 template <int D>
 __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &sm)
@@ -201,20 +202,19 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
     constexpr int TK = SimtCfg<D>::TK;
     constexpr int NSTAGE = SimtCfg<D>::NSTAGE;
     const uint64_t pol = l2_evict_first_policy();
-    ItemCursor cur, ahead;
-    cur.init();
-    ahead.init();
+    SegCursor cur;
+    cur.init(p, sm.range);
     WorkItem it, nx;
     uint32_t T = 0;
-    uint32_t j = 0;  // item counter of this CTA
-    int64_t i = blockIdx.x;
-    uint32_t q_issued = 0;  // items whose query copy was started
-    bool have = cur.seek(p, i, it);
+    uint32_t j = 0;  // segment counter of this CTA
+    uint32_t q_issued = 0;  // segments whose query copy was started
+    bool have = cur.next(p, it);
     if (have && producer_q<D>(p, sm, it, 0, pol))
         q_issued = 1;
     int32_t page_next = have ? __ldg(p.table + (int64_t)it.s * p.table_stride + it.key0 / p.P) : 0;
     while (have && !sm.abort_flag) {
-        const bool have_nx = ahead.seek(p, i + gridDim.x, nx);
+        SegCursor ahead = cur;
+        const bool have_nx = ahead.next(p, nx);
         if (have_nx && producer_q<D>(p, sm, nx, j + 1, pol))
             q_issued = j + 2;
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
@@ -251,7 +251,6 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
         have = have_nx;
         it = nx;
         cur = ahead;
-        i += gridDim.x;
         ++j;
     }
     if (sm.abort_flag) {
@@ -291,14 +290,14 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
     const int li = lane % LG;
     const float NEG_INF = -__int_as_float(0x7f800000);
 
-    ItemCursor cur;
-    cur.init();
+    SegCursor cur;
+    cur.init(p, sm.range);
     WorkItem it;
-    uint32_t T0 = 0;  // CTA tile index of the item's first tile
+    uint32_t T0 = 0;  // CTA tile index of the segment's first tile
     uint32_t j = 0;
 
-    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
-        // --- this item's query rows: packed bf16 pairs in registers --------
+    for (; cur.next(p, it); ++j) {
+        // --- this segment's query rows: packed bf16 pairs in registers --------
         uint32_t qh[kR][CPL * 4];
         int lim[kR];
         {
@@ -508,7 +507,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
             for (int r = 0; r < kR; ++r)
                 l_row[r] = __shfl_sync(0xffffffffu, lr, r);
         }
-        // the slot is free once the previous item's combine is done
+        // the slot is free once the previous segment's combine is done
         (void)wait_or_abort(sm, &sm.w_free, (j & 1u) ^ 1u, p.flags, kWaitFree);
         if (lane == 0) {
 #pragma unroll
@@ -567,19 +566,19 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 continue;
             float *dst;
             float scale_out;
-            if (it.nc == 1) {
+            if (it.fin) {
                 const int wr = m / p.G;
                 const int h = it.kh * p.G + (m - wr * p.G);
                 dst = p.out + (((size_t)it.s * p.W + wr) * p.Hq + h) * D;
                 scale_out = 1.f / lstar;
             } else {
                 float *slot =
-                    p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(p.RB * (D + 2));
+                    p.part + (size_t)it.slot * (p.SR * (D + 2));
                 dst = slot + (size_t)r * D;
                 scale_out = 1.f;
                 if (lane == 0) {
-                    slot[(size_t)p.RB * D + r] = mstar;
-                    slot[(size_t)p.RB * D + p.RB + r] = lstar;
+                    slot[(size_t)p.SR * D + r] = mstar;
+                    slot[(size_t)p.SR * D + p.SR + r] = lstar;
                 }
             }
 #pragma unroll
@@ -627,6 +626,8 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == SimtCfg<D>::NCW)
+        find_range(p, sm.range, lane);
     __syncthreads();
     if (warp == SimtCfg<D>::NCW) {
         if (lane == 0)

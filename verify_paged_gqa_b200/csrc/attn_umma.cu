@@ -21,7 +21,7 @@
 //              (so no NaN from unused slots reaches the MMA: 0 * NaN = NaN).
 //   warps 2-5  softmax (one query row per thread, the row's TMEM lane): write
 //              the row's query into the swizzled Q tile at the start of each
-//              item; per tile, read the S row from TMEM, select masked
+//              segment; per tile, read the S row from TMEM, select masked
 //              positions to -inf, update the running max m and sum l in log2
 //              units, and write P into TMEM as two bf16 parts (P = hi + lo,
 //              each the truncated upper half of a float, so the PV product
@@ -30,7 +30,7 @@
 //              read their A operand from there, so shared memory holds only
 //              the K/V ring (7 stages).  O in TMEM is rescaled only when the row max
 //              grows by more than 2^8 (exact: the final O / l does not depend
-//              on the reference max).  At the end of the item the row is
+//              on the reference max).  At the end of the segment the row is
 //              normalised and stored, or left as a partial for the merge.
 #include "launch.cuh"
 #include "plan.cuh"
@@ -53,12 +53,13 @@ struct UmmaSmem {
     alignas(1024) uint8_t kv[NST][4][UN * 128];
     uint64_t kv_full[NST];
     uint64_t kv_empty[NST];
-    uint64_t q_full;       // softmax warps wrote the item's Q tile
-    uint64_t q_free;       // the item's last QK MMA is done with Q
+    uint64_t q_full;       // softmax warps wrote the segment's Q tile
+    uint64_t q_free;       // the segment's last QK MMA is done with Q
     uint64_t s_full[2];
     uint64_t p_full[2];    // softmax warps wrote P into buffer b
     uint64_t o_done[2];    // the PV reading P buffer b finished (and every MMA before it)
     uint64_t fin;          // every MMA this CTA issued has completed
+    CtaRange range;        // this CTA's tiles
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -90,16 +91,15 @@ __device__ __forceinline__ void umma_producer(const UmmaArgs &a, UmmaSmem &sm)
 {
     const AttnParams &p = a.p;
     const uint64_t pol = l2_evict_first_policy();
-    ItemCursor cur, ahead;
-    cur.init();
-    ahead.init();
+    SegCursor cur;
+    cur.init(p, sm.range);
     WorkItem it, nx;
     uint32_t T = 0;
-    int64_t i = blockIdx.x;
-    bool have = cur.seek(p, i, it);
+    bool have = cur.next(p, it);
     int32_t page_next = have ? __ldg(p.table + (int64_t)it.s * p.table_stride + it.key0 / p.P) : 0;
     while (have && !sm.abort_flag) {
-        const bool have_nx = ahead.seek(p, i + gridDim.x, nx);
+        SegCursor ahead = cur;
+        const bool have_nx = ahead.next(p, nx);
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
         const int lp_end = (it.key1 + p.P - 1) / p.P;
         for (int lp = it.key0 / p.P; lp < lp_end && !sm.abort_flag; ++lp) {
@@ -132,7 +132,7 @@ __device__ __forceinline__ void umma_producer(const UmmaArgs &a, UmmaSmem &sm)
         }
         have = have_nx;
         it = nx;
-        i += gridDim.x;
+        cur = ahead;
     }
     if (sm.abort_flag) {
         const uint32_t n = T < (uint32_t)NST ? T : (uint32_t)NST;
@@ -180,12 +180,12 @@ __device__ __forceinline__ void umma_issuer(const UmmaArgs &a, UmmaSmem &sm)
     constexpr uint32_t kHalf = UN * 128;          // one [UN][64] bf16 box
     constexpr uint32_t kStageBytes = 4 * kHalf;
 
-    ItemCursor cur;
-    cur.init();
+    SegCursor cur;
+    cur.init(p, sm.range);
     WorkItem it;
     uint32_t T0 = 0, j = 0;
     bool ok = true;
-    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
+    for (; cur.next(p, it); ++j) {
         const int ntiles = (it.key1 - it.key0 + UN - 1) / UN;
         ok = ok && uwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
         tc_fence_after();
@@ -260,11 +260,11 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
     const uint32_t tO = lane_base + kColO;
     const float NEG_INF = -__int_as_float(0x7f800000);
 
-    ItemCursor cur;
-    cur.init();
+    SegCursor cur;
+    cur.init(p, sm.range);
     WorkItem it;
     uint32_t j = 0, tt = 0;
-    for (int64_t i = blockIdx.x; cur.seek(p, i, it); i += gridDim.x, ++j) {
+    for (; cur.next(p, it); ++j) {
         const int m = it.b * MR + row;
         const bool live = lane_rows && m < p.M;
         const int lim = row_lim(p, it.len, m);
@@ -273,7 +273,7 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
         // --- the row's query into the swizzled Q tile ----------------------
         bool ok;
         {
-            // load the row first (overlaps the wait for the previous item's last QK)
+            // load the row first (overlaps the wait for the previous segment's last QK)
             const int mm = min(m, p.M - 1);
             const int wr = mm / p.G;
             const int h = it.kh * p.G + (mm - wr * p.G);
@@ -404,7 +404,7 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
             if (lane == 0)
                 mbar_arrive(&sm.p_full[u & 1]);
         }
-        // --- the item's last PV, then the row's result ----------------------
+        // --- the segment's last PV, then the row's result ----------------------
         const uint32_t ulast = tt + ntiles - 1;
         ok = uwait(sm, &sm.o_done[ulast & 1], (ulast >> 1) & 1u, p.flags, kWaitEmpty) && ok;
         tc_fence_after();
@@ -412,17 +412,17 @@ __device__ __forceinline__ void umma_softmax(const UmmaArgs &a, UmmaSmem &sm, in
         float *dst = nullptr;
         float sc = 1.f;
         if (write) {
-            if (it.nc == 1) {
+            if (it.fin) {
                 const int wr = m / p.G;
                 const int h = it.kh * p.G + (m - wr * p.G);
                 dst = p.out + (((size_t)it.s * p.W + wr) * p.Hq + h) * UD;
                 sc = 1.f / l_run;
             } else {
                 float *slot =
-                    p.part + part_slot(p, it.s, it.kh, it.b, it.c) * (size_t)(p.RB * (UD + 2));
+                    p.part + (size_t)it.slot * (p.SR * (UD + 2));
                 dst = slot + (size_t)row * UD;
-                slot[(size_t)p.RB * UD + row] = m_run;
-                slot[(size_t)p.RB * UD + p.RB + row] = l_run;
+                slot[(size_t)p.SR * UD + row] = m_run;
+                slot[(size_t)p.SR * UD + p.SR + row] = l_run;
             }
         }
 #pragma unroll 1
@@ -467,6 +467,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) attn_umma_kernel(const __grid
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    if (warp == 0)
+        find_range(a.p, sm.range, lane);
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr(&sm.tmem_base)), "r"(kTmemCols)

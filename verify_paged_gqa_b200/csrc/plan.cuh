@@ -1,21 +1,32 @@
-// plan.cuh -- how one attention call is cut into work items.
+// plan.cuh -- how one attention call is cut into work (stream-K).
 //
-// A unit is (stream s, KV head kh).  Its M = G * W query rows (W window
-// rows times the G query heads of the group, row m = r * G + g) are cut into
-// row blocks of RB rows, and the keys a row block can see are cut into
-// chunks of CH positions (CH a multiple of the page size, fixed by host
-// arguments only).  One work item = (s, kh, row block b, chunk c).  Items are
-// numbered stream by stream, then KV head, row block, chunk; persistent CTAs
-// take items round-robin.  A row block with one chunk is finished by its
-// item; otherwise every item leaves a partial (unnormalised O, running max,
-// running sum) in a fixed slot of the workspace and the merge kernel
-// combines them in chunk order.  Which CTA runs an item never changes its
-// arithmetic, so results depend only on positions, lens and host arguments.
+// A unit is (stream s, KV head kh, row block b): its RB query rows (of the
+// M = G * W rows of (s, kh); row m = r * G + g) and the keys they can see,
+// [0, block_lim).  Those keys are cut into tiles of kTile positions.  The
+// launch's units are laid end to end -- stream by stream, then KV head, then
+// row block -- and their tiles are split evenly over the persistent CTAs:
+// with T tiles in all and G CTAs, CTA c takes tiles [c T / G, (c + 1) T / G).
+// The split is computed on the device from the streams' actual lengths, so
+// every CTA gets the same work (to one tile) whatever the length mix, and a
+// captured graph stays valid as the lengths grow.
+//
+// A CTA's range meets a run of units; each meeting is a segment.  A segment
+// that covers its whole unit finishes the unit's rows itself.  Otherwise it
+// leaves a partial (unnormalised O, running max, running sum) in one of the
+// CTA's two workspace slots: slot 2c for a segment that starts at the CTA's
+// first tile, 2c + 1 for one that ends at its last (a CTA range meets at most
+// two units partially).  The merge kernel finds a split unit's segments from
+// the same arithmetic and combines them in position order.  A unit's result
+// therefore depends on the lengths of the call's streams and the grid size
+// (never on the page table, nor on run-to-run timing).
 #pragma once
 
 #include "common.cuh"
 
 namespace tfp {
+
+constexpr int kTile = 128;     // positions per scheduling tile
+constexpr int kMaxCtas = 1024; // persistent CTAs of a partial kernel, at most
 
 __host__ __device__ __forceinline__ bool len_ok(const AttnParams &p, int len)
 {
@@ -35,75 +46,161 @@ __host__ __device__ __forceinline__ int row_lim(const AttnParams &p, int len, in
     return len - p.W + min(m, p.M - 1) / p.G + 1;
 }
 
-__host__ __device__ __forceinline__ int block_chunks(const AttnParams &p, int len, int b)
+__host__ __device__ __forceinline__ int unit_tiles(const AttnParams &p, int len, int b)
 {
-    return (block_lim(p, len, b) + p.CH - 1) / p.CH;
+    return (block_lim(p, len, b) + kTile - 1) / kTile;
 }
 
-__host__ __device__ __forceinline__ int64_t part_slot(const AttnParams &p, int s, int kh, int b,
-                                                      int c)
-{
-    return (((int64_t)s * p.Hkv + kh) * p.n_rblk + b) * p.max_chunks + c;
-}
-
-__device__ __forceinline__ int stream_items(const AttnParams &p, int len)
+// Tiles of one KV head of a stream (all its row blocks); 0 for a length out
+// of range (those streams are skipped and reported by the merge kernel).
+__host__ __device__ __forceinline__ int64_t head_tiles(const AttnParams &p, int len)
 {
     if (!len_ok(p, len))
         return 0;
-    int n = 0;
+    int64_t n = 0;
     for (int b = 0; b < p.n_rblk; ++b)
-        n += block_chunks(p, len, b);
-    return n * p.Hkv;
+        n += unit_tiles(p, len, b);
+    return n;
+}
+
+// First tile of CTA c's range, and the CTA whose range holds tile g.
+__host__ __device__ __forceinline__ int64_t range_start(int64_t tot, int c, int n_cta)
+{
+    return tot * c / n_cta;
+}
+
+__host__ __device__ __forceinline__ int cta_of(int64_t g, int64_t tot, int n_cta)
+{
+    return static_cast<int>((g * n_cta + n_cta - 1) / tot);
+}
+
+// This CTA's range, found by warp 0 at kernel start.
+struct CtaRange {
+    long long g0, g1;   // tiles [g0, g1) of the launch
+    long long off0;     // g0's offset inside stream s0
+    int s0;             // stream holding tile g0 (S when the range is empty)
+    int pad;
+};
+
+// Run by one whole warp.  Two passes over the streams' lengths, 32 at a
+// time: the total, then the stream holding the CTA's first tile.  CTA 0 also
+// records every stream's first tile and the total in the workspace for the
+// merge kernel.
+__device__ __forceinline__ void find_range(const AttnParams &p, CtaRange &out, int lane)
+{
+    long long tot = 0;
+    for (int s = lane; s < p.S; s += 32)
+        tot += p.Hkv * head_tiles(p, __ldg(p.lens + s));
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1)
+        tot += __shfl_xor_sync(0xffffffffu, tot, k);
+    const long long g0 = range_start(tot, blockIdx.x, gridDim.x);
+    const long long g1 = range_start(tot, blockIdx.x + 1, gridDim.x);
+    const bool writer = blockIdx.x == 0;
+    int s0 = p.S;
+    long long off0 = 0, base = 0;
+    for (int c0 = 0; c0 < p.S && (writer || (g0 < g1 && s0 == p.S)); c0 += 32) {
+        const int s = c0 + lane;
+        const long long t = s < p.S ? p.Hkv * head_tiles(p, __ldg(p.lens + s)) : 0;
+        long long incl = t;
+#pragma unroll
+        for (int k = 1; k < 32; k <<= 1) {
+            const long long v = __shfl_up_sync(0xffffffffu, incl, k);
+            if (lane >= k)
+                incl += v;
+        }
+        const long long excl = base + incl - t;
+        if (writer && s < p.S)
+            p.first_tile[s] = excl;
+        const unsigned hit = __ballot_sync(0xffffffffu, t > 0 && excl <= g0 && g0 < excl + t);
+        if (hit != 0 && s0 == p.S) {
+            const int L = __ffs(hit) - 1;
+            s0 = c0 + L;
+            off0 = g0 - __shfl_sync(0xffffffffu, excl, L);
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (writer && lane == 0)
+        *p.total_tiles = tot;
+    if (lane == 0) {
+        out.g0 = g0;
+        out.g1 = g1;
+        out.off0 = off0;
+        out.s0 = g0 < g1 ? s0 : p.S;
+    }
 }
 
 struct WorkItem {
-    int s, kh, b, c, nc, len;
-    int key0, key1;  // positions [key0, key1) this item reads
+    int s, kh, b, len;
+    int key0, key1;  // positions [key0, key1) this segment reads
+    bool fin;        // covers the whole unit: write the rows' outputs
+    int slot;        // partial slot otherwise
 };
 
-// Walks the item numbering; seek() must be called with non-decreasing i.
-struct ItemCursor {
-    int s;
-    int64_t base;
-    int cnt;
-    int len;
+// Walks this CTA's segments in order; each role of a CTA keeps its own.
+struct SegCursor {
+    int s, kh, b, off, len;
+    long long left;
+    bool first;
 
-    __device__ __forceinline__ void init()
+    __device__ __forceinline__ void init(const AttnParams &p, const CtaRange &r)
     {
-        s = -1;
-        base = 0;
-        cnt = 0;
+        left = r.g1 - r.g0;
+        first = true;
+        s = r.s0;
+        kh = b = off = 0;
         len = 0;
+        if (left <= 0 || s >= p.S) {
+            left = 0;
+            return;
+        }
+        len = __ldg(p.lens + s);
+        const long long ht = head_tiles(p, len);
+        kh = static_cast<int>(r.off0 / ht);
+        int rem = static_cast<int>(r.off0 - kh * ht);
+        for (;;) {
+            const int tu = unit_tiles(p, len, b);
+            if (rem < tu)
+                break;
+            rem -= tu;
+            ++b;
+        }
+        off = rem;
     }
 
-    __device__ __forceinline__ bool seek(const AttnParams &p, int64_t i, WorkItem &w)
+    __device__ __forceinline__ bool next(const AttnParams &p, WorkItem &w)
     {
-        while (i >= base + cnt) {
-            base += cnt;
-            ++s;
-            if (s >= p.S)
-                return false;
-            len = __ldg(p.lens + s);
-            cnt = stream_items(p, len);
-        }
-        const int r = static_cast<int>(i - base);
-        const int per_kh = cnt / p.Hkv;
+        if (left <= 0)
+            return false;
+        const int tu = unit_tiles(p, len, b);
+        const int n = static_cast<int>(min((long long)(tu - off), left));
         w.s = s;
-        w.len = len;
-        w.kh = r / per_kh;
-        int r2 = r - w.kh * per_kh;
-        int b = 0;
-        for (; b < p.n_rblk - 1; ++b) {
-            const int nc = block_chunks(p, len, b);
-            if (r2 < nc)
-                break;
-            r2 -= nc;
-        }
+        w.kh = kh;
         w.b = b;
-        w.c = r2;
-        w.nc = block_chunks(p, len, b);
-        w.key0 = r2 * p.CH;
-        w.key1 = min(w.key0 + p.CH, block_lim(p, len, b));
+        w.len = len;
+        w.key0 = off * kTile;
+        w.key1 = min((off + n) * kTile, block_lim(p, len, b));
+        w.fin = off == 0 && n == tu;
+        w.slot = w.fin ? -1 : 2 * static_cast<int>(blockIdx.x) + (first ? 0 : 1);
+        first = false;
+        left -= n;
+        off += n;
+        if (left > 0) {
+            // the next unit with tiles
+            off = 0;
+            if (++b == p.n_rblk) {
+                b = 0;
+                if (++kh == p.Hkv) {
+                    kh = 0;
+                    do {
+                        ++s;
+                        len = s < p.S ? __ldg(p.lens + s) : 0;
+                    } while (s < p.S && head_tiles(p, len) == 0);
+                    if (s >= p.S)
+                        left = 0;
+                }
+            }
+        }
         return true;
     }
 };

@@ -58,36 +58,22 @@ int check_pool_streams(const tf_kv_pool *pool, const tf_streams *st)
 
 enum class Kernel { kSimt, kUmma, kPm };
 
+// Workspace: the 256-byte header (status word, wait site, the launch's tile
+// count at byte 64), each stream's first tile (int64), then two partial slots
+// per CTA of min(RB, M) rows x (D + 2) floats.
+constexpr size_t kWsTotalOffset = 64;
+
+size_t ws_part_offset(int S)
+{
+    return kWsHeaderBytes + (((size_t)S * 8 + 255) / 256) * 256;
+}
+
 struct Plan {
     AttnParams p;
     int grid;
     size_t ws_bytes;
     Kernel kernel;  // which partial kernel runs the call
 };
-
-// Chunk length in pages: the one that minimises the busiest CTA's pages
-// (items are dealt round-robin to one CTA per SM) plus the partials' write
-// and read traffic, assuming every stream at max_len.
-int choose_chunk_pages(int64_t units, int pages_max, int grid, double partial_pages_per_item)
-{
-    int best = 1;
-    double best_cost = 1e300;
-    const int cap = pages_max < 64 ? pages_max : 64;
-    for (int cp = 1; cp <= cap; ++cp) {
-        const int64_t per_unit = (pages_max + cp - 1) / cp;
-        const int64_t items = units * per_unit;
-        const int64_t rounds = (items + grid - 1) / grid;
-        double cost = (double)rounds * cp;
-        if (per_unit > 1)
-            cost += (double)items * partial_pages_per_item / grid;
-        cost += 0.02 * (double)rounds;  // per-item fixed cost (pipeline turn, combine)
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = cp;
-        }
-    }
-    return best;
-}
 
 int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t rows,
               int32_t rows_max, Plan *plan)
@@ -138,21 +124,17 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
         }
     }
     p.n_rblk = static_cast<int32_t>((M + p.RB - 1) / p.RB);
+    p.SR = static_cast<int32_t>(M < p.RB ? M : p.RB);
 
-    const int pages_max = (st->max_len + p.P - 1) / p.P;
-    const int64_t units = (int64_t)p.S * p.Hkv * p.n_rblk;
-    const int grid_cap = sms;  // one persistent CTA per SM
-    const double partial_bytes = 2.0 * p.RB * (p.D + 2) * 4.0;
-    const double page_bytes = 2.0 * p.P * p.D * 2.0;
-    const int cp = choose_chunk_pages(units > 0 ? units : 1, pages_max, grid_cap,
-                                      partial_bytes / page_bytes);
-    p.CH = cp * p.P;
-    p.max_chunks = (st->max_len + p.CH - 1) / p.CH;
-    const int64_t items_max = units * p.max_chunks;
-    plan->grid = static_cast<int>(items_max < grid_cap ? (items_max > 0 ? items_max : 1) : grid_cap);
-    plan->ws_bytes = kWsHeaderBytes;
-    if (p.max_chunks > 1)
-        plan->ws_bytes += (size_t)units * p.max_chunks * p.RB * (p.D + 2) * sizeof(float);
+    // One persistent CTA per SM, but no more than the tiles the call can
+    // have with every stream at max_len (the device splits the actual ones).
+    const int64_t tiles_max = (int64_t)p.S * p.Hkv * head_tiles(p, st->max_len);
+    int64_t grid = sms < kMaxCtas ? sms : kMaxCtas;
+    if (tiles_max < grid)
+        grid = tiles_max > 0 ? tiles_max : 1;
+    plan->grid = static_cast<int>(grid);
+    p.n_cta = plan->grid;
+    plan->ws_bytes = ws_part_offset(p.S) + (size_t)2 * plan->grid * p.SR * (p.D + 2) * sizeof(float);
     return TF_OK;
 }
 
@@ -179,8 +161,11 @@ int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32
     p.lens = st->lens;
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.out = out;
-    p.flags = static_cast<uint32_t *>(ws);
-    p.part = reinterpret_cast<float *>(static_cast<char *>(ws) + kWsHeaderBytes);
+    char *wsb = static_cast<char *>(ws);
+    p.flags = reinterpret_cast<uint32_t *>(wsb);
+    p.total_tiles = reinterpret_cast<long long *>(wsb + kWsTotalOffset);
+    p.first_tile = reinterpret_cast<long long *>(wsb + kWsHeaderBytes);
+    p.part = reinterpret_cast<float *>(wsb + ws_part_offset(p.S));
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
