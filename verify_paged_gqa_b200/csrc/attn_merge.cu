@@ -10,9 +10,8 @@
 // The maximum and the sum of l are warp-shuffle reductions; the O sum runs
 // in segment (position) order, so the result is the same on every run.
 //
-// The segments of a unit split across CTAs are found from the tile split
-// (plan.cuh): the CTAs whose ranges meet the unit's tiles [U0, U1), in
-// order.  One block per (stream, KV head, row block, group of up to 8 rows);
+// The segments of a unit split across CTAs are found from the work split
+// (plan.cuh): the CTAs whose ranges meet the unit's real tiles, in order.  One block per (stream, KV head, row block, group of up to 8 rows);
 // one warp per row.  The weighted sum loads several segments' rows before
 // using them, so the loads of a round overlap.  Streams whose length is out
 // of range get NaN rows (and the status bit).
@@ -61,25 +60,44 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
         }
         return;
     }
-    // the unit's tiles [U0, U1) and the CTAs that met them
-    const long long tot = *p.total_tiles;
-    long long U0 = p.first_tile[s] + kh * head_tiles(p, len);
-    for (int bb = 0; bb < b; ++bb)
-        U0 += unit_tiles(p, len, bb);
-    const long long U1 = U0 + unit_tiles(p, len, b);
-    const int c_lo = cta_of(U0, tot, p.n_cta);
-    const int c_hi = cta_of(U1 - 1, tot, p.n_cta);
-    if (c_lo == c_hi)
-        return;  // one segment covered the unit and wrote the rows itself
-    const int nseg = min(c_hi - c_lo + 1, kMaxCtas);
-    for (int k = threadIdx.x; k < nseg; k += blockDim.x) {
-        const int c = c_lo + k;
-        const long long a0 = range_start(tot, c, p.n_cta);
-        const long long a1 = range_start(tot, c + 1, p.n_cta);
-        // the first CTA's segment is its last unless its range starts at U0
-        slots[k] = a0 == a1 ? -1 : (k == 0 && a0 < U0) ? 2 * c + 1 : 2 * c;
+    // the unit's tiles [U0, U1) and the CTAs that met them: warp 0 works them
+    // out once for the block (lanes split the row blocks)
+    __shared__ int nseg_sh;
+    if (warp == 0) {
+        long long hw = 0, before = 0;
+        for (int bb = lane; bb < p.n_rblk; bb += 32) {
+            const int t = unit_work(p, len, bb);
+            hw += t;
+            if (bb < b)
+                before += t;
+        }
+#pragma unroll
+        for (int k = 16; k >= 1; k >>= 1) {
+            hw += __shfl_xor_sync(0xffffffffu, hw, k);
+            before += __shfl_xor_sync(0xffffffffu, before, k);
+        }
+        const long long tot = *p.total_tiles;
+        // the unit's work [U0, U1): entry tiles, then its tiles from U0 + VT
+        const long long U0 = p.first_tile[s] + kh * hw + before;
+        const long long U1 = U0 + unit_work(p, len, b);
+        const int c_lo = cta_of(U0 + p.VT, tot, p.n_cta);
+        const int c_hi = cta_of(U1 - 1, tot, p.n_cta);
+        const int n = min(c_hi - c_lo + 1, kMaxCtas);
+        for (int k = lane; k < n; k += 32) {
+            const int c = c_lo + k;
+            const long long a0 = range_start(tot, c, p.n_cta);
+            const long long a1 = range_start(tot, c + 1, p.n_cta);
+            // the first CTA's segment is its last unless its range starts at U0
+            slots[k] = a0 == a1 ? -1 : (k == 0 && a0 < U0) ? 2 * c + 1 : 2 * c;
+        }
+        // one segment covered the unit and wrote the rows itself
+        if (lane == 0)
+            nseg_sh = c_lo == c_hi ? 0 : n;
     }
     __syncthreads();
+    const int nseg = nseg_sh;
+    if (nseg == 0)
+        return;
     const size_t slot_floats = (size_t)p.SR * (D + 2);
 
     for (int m = m0 + warp; m < m1; m += nwarps) {

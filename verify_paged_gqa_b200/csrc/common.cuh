@@ -49,9 +49,10 @@ struct AttnParams {
     int32_t Hq, G, W, M;        // M = G * W query rows per (stream, KV head)
     int32_t RB, n_rblk;         // rows per row block, row blocks per (stream, KV head)
     int32_t SR;                 // rows per partial slot: min(RB, M)
-    int32_t n_cta;              // persistent CTAs of the partial kernel (the tile split)
-    long long *first_tile;      // workspace: each stream's first tile in the launch
-    long long *total_tiles;     // workspace: tiles of the launch
+    int32_t n_cta;              // persistent CTAs of the partial kernel (the work split)
+    int32_t VT;                 // entry tiles of work in front of every unit
+    long long *first_tile;      // workspace: where each stream's work starts in the launch
+    long long *total_tiles;     // workspace: work tiles of the launch
     float scale_log2;           // scale * log2(e): scores are kept in log2 units
 };
 

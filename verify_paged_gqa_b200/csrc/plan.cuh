@@ -4,11 +4,15 @@
 // M = G * W rows of (s, kh); row m = r * G + g) and the keys they can see,
 // [0, block_lim).  Those keys are cut into tiles of kTile positions.  The
 // launch's units are laid end to end -- stream by stream, then KV head, then
-// row block -- and their tiles are split evenly over the persistent CTAs:
-// with T tiles in all and G CTAs, CTA c takes tiles [c T / G, (c + 1) T / G).
-// The split is computed on the device from the streams' actual lengths, so
-// every CTA gets the same work (to one tile) whatever the length mix, and a
-// captured graph stays valid as the lengths grow.
+// row block -- and their work is split evenly over the persistent CTAs.  A
+// unit's work is its tiles plus VT "entry" tiles in front of them that hold
+// no positions: they stand for what a CTA pays to start a unit (its query
+// rows, the pipeline filling again, one more epilogue), so a CTA whose range
+// crosses into a new unit gets that many fewer real tiles.  With T work
+// tiles in all and G CTAs, CTA c takes [c T / G, (c + 1) T / G).  The split
+// is computed on the device from the streams' actual lengths, so every CTA
+// gets the same work whatever the length mix, and a captured graph stays
+// valid as the lengths grow.
 //
 // A CTA's range meets a run of units; each meeting is a segment.  A segment
 // that covers its whole unit finishes the unit's rows itself.  Otherwise it
@@ -51,19 +55,25 @@ __host__ __device__ __forceinline__ int unit_tiles(const AttnParams &p, int len,
     return (block_lim(p, len, b) + kTile - 1) / kTile;
 }
 
-// Tiles of one KV head of a stream (all its row blocks); 0 for a length out
+// Work of a unit: its entry tiles, then its tiles.
+__host__ __device__ __forceinline__ int unit_work(const AttnParams &p, int len, int b)
+{
+    return p.VT + unit_tiles(p, len, b);
+}
+
+// Work of one KV head of a stream (all its row blocks); 0 for a length out
 // of range (those streams are skipped and reported by the merge kernel).
-__host__ __device__ __forceinline__ int64_t head_tiles(const AttnParams &p, int len)
+__host__ __device__ __forceinline__ int64_t head_work(const AttnParams &p, int len)
 {
     if (!len_ok(p, len))
         return 0;
     int64_t n = 0;
     for (int b = 0; b < p.n_rblk; ++b)
-        n += unit_tiles(p, len, b);
+        n += unit_work(p, len, b);
     return n;
 }
 
-// First tile of CTA c's range, and the CTA whose range holds tile g.
+// First work tile of CTA c's range, and the CTA whose range holds work tile g.
 __host__ __device__ __forceinline__ int64_t range_start(int64_t tot, int c, int n_cta)
 {
     return tot * c / n_cta;
@@ -76,21 +86,21 @@ __host__ __device__ __forceinline__ int cta_of(int64_t g, int64_t tot, int n_cta
 
 // This CTA's range, found by warp 0 at kernel start.
 struct CtaRange {
-    long long g0, g1;   // tiles [g0, g1) of the launch
+    long long g0, g1;   // work tiles [g0, g1) of the launch
     long long off0;     // g0's offset inside stream s0
     int s0;             // stream holding tile g0 (S when the range is empty)
     int pad;
 };
 
 // Run by one whole warp.  Two passes over the streams' lengths, 32 at a
-// time: the total, then the stream holding the CTA's first tile.  CTA 0 also
-// records every stream's first tile and the total in the workspace for the
-// merge kernel.
+// time: the total work, then the stream holding the CTA's first work tile.
+// CTA 0 also records where every stream's work starts and the total in the
+// workspace for the merge kernel.
 __device__ __forceinline__ void find_range(const AttnParams &p, CtaRange &out, int lane)
 {
     long long tot = 0;
     for (int s = lane; s < p.S; s += 32)
-        tot += p.Hkv * head_tiles(p, __ldg(p.lens + s));
+        tot += p.Hkv * head_work(p, __ldg(p.lens + s));
 #pragma unroll
     for (int k = 16; k >= 1; k >>= 1)
         tot += __shfl_xor_sync(0xffffffffu, tot, k);
@@ -101,7 +111,7 @@ __device__ __forceinline__ void find_range(const AttnParams &p, CtaRange &out, i
     long long off0 = 0, base = 0;
     for (int c0 = 0; c0 < p.S && (writer || (g0 < g1 && s0 == p.S)); c0 += 32) {
         const int s = c0 + lane;
-        const long long t = s < p.S ? p.Hkv * head_tiles(p, __ldg(p.lens + s)) : 0;
+        const long long t = s < p.S ? p.Hkv * head_work(p, __ldg(p.lens + s)) : 0;
         long long incl = t;
 #pragma unroll
         for (int k = 1; k < 32; k <<= 1) {
@@ -137,9 +147,10 @@ struct WorkItem {
     int slot;        // partial slot otherwise
 };
 
-// Walks this CTA's segments in order; each role of a CTA keeps its own.
+// Walks this CTA's segments in order; each role of a CTA keeps its own.  A
+// part of the range that holds only a unit's entry tiles yields no segment.
 struct SegCursor {
-    int s, kh, b, off, len;
+    int s, kh, b, off, len;   // off: work tiles of unit (s, kh, b) already passed
     long long left;
     bool first;
 
@@ -155,14 +166,14 @@ struct SegCursor {
             return;
         }
         len = __ldg(p.lens + s);
-        const long long ht = head_tiles(p, len);
-        kh = static_cast<int>(r.off0 / ht);
-        int rem = static_cast<int>(r.off0 - kh * ht);
+        const long long hw = head_work(p, len);
+        kh = static_cast<int>(r.off0 / hw);
+        int rem = static_cast<int>(r.off0 - kh * hw);
         for (;;) {
-            const int tu = unit_tiles(p, len, b);
-            if (rem < tu)
+            const int wu = unit_work(p, len, b);
+            if (rem < wu)
                 break;
-            rem -= tu;
+            rem -= wu;
             ++b;
         }
         off = rem;
@@ -170,38 +181,44 @@ struct SegCursor {
 
     __device__ __forceinline__ bool next(const AttnParams &p, WorkItem &w)
     {
-        if (left <= 0)
-            return false;
-        const int tu = unit_tiles(p, len, b);
-        const int n = static_cast<int>(min((long long)(tu - off), left));
-        w.s = s;
-        w.kh = kh;
-        w.b = b;
-        w.len = len;
-        w.key0 = off * kTile;
-        w.key1 = min((off + n) * kTile, block_lim(p, len, b));
-        w.fin = off == 0 && n == tu;
-        w.slot = w.fin ? -1 : 2 * static_cast<int>(blockIdx.x) + (first ? 0 : 1);
-        first = false;
-        left -= n;
-        off += n;
-        if (left > 0) {
-            // the next unit with tiles
-            off = 0;
-            if (++b == p.n_rblk) {
-                b = 0;
-                if (++kh == p.Hkv) {
-                    kh = 0;
-                    do {
-                        ++s;
-                        len = s < p.S ? __ldg(p.lens + s) : 0;
-                    } while (s < p.S && head_tiles(p, len) == 0);
-                    if (s >= p.S)
-                        left = 0;
+        while (left > 0) {
+            const int wu = unit_work(p, len, b);
+            const int n = static_cast<int>(min((long long)(wu - off), left));
+            const int t0 = max(off - p.VT, 0), t1 = max(off + n - p.VT, 0);  // real tiles
+            const bool emit = t1 > t0;
+            if (emit) {
+                w.s = s;
+                w.kh = kh;
+                w.b = b;
+                w.len = len;
+                w.key0 = t0 * kTile;
+                w.key1 = min(t1 * kTile, block_lim(p, len, b));
+                w.fin = t0 == 0 && t1 == wu - p.VT;
+                w.slot = w.fin ? -1 : 2 * static_cast<int>(blockIdx.x) + (first ? 0 : 1);
+                first = false;
+            }
+            left -= n;
+            off += n;
+            if (left > 0) {
+                // the next unit with work
+                off = 0;
+                if (++b == p.n_rblk) {
+                    b = 0;
+                    if (++kh == p.Hkv) {
+                        kh = 0;
+                        do {
+                            ++s;
+                            len = s < p.S ? __ldg(p.lens + s) : 0;
+                        } while (s < p.S && head_work(p, len) == 0);
+                        if (s >= p.S)
+                            left = 0;
+                    }
                 }
             }
+            if (emit)
+                return true;
         }
-        return true;
+        return false;
     }
 };
 

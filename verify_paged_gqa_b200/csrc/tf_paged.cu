@@ -68,6 +68,15 @@ size_t ws_part_offset(int S)
     return kWsHeaderBytes + (((size_t)S * 8 + 255) / 256) * 256;
 }
 
+// Entry tiles per unit (plan.cuh), measured: at head dim 512 a unit start
+// costs about 8 tiles' worth of streaming (the ring holds less than one
+// tile, so the pipeline drains and refills); the CUDA-core decode kernel's
+// segment starts overlap with its deep ring and cost nothing measurable.
+constexpr int kEntryPm512 = 8;
+constexpr int kEntryPm128 = 4;
+constexpr int kEntryUmma = 4;
+constexpr int kEntrySimt = 0;
+
 struct Plan {
     AttnParams p;
     int grid;
@@ -126,9 +135,13 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     p.n_rblk = static_cast<int32_t>((M + p.RB - 1) / p.RB);
     p.SR = static_cast<int32_t>(M < p.RB ? M : p.RB);
 
-    // One persistent CTA per SM, but no more than the tiles the call can
-    // have with every stream at max_len (the device splits the actual ones).
-    const int64_t tiles_max = (int64_t)p.S * p.Hkv * head_tiles(p, st->max_len);
+    // Entry cost of a unit, in tiles: what starting one more unit costs a
+    // CTA relative to streaming one tile of it (measured per kernel).
+    p.VT = plan->kernel == Kernel::kPm ? (p.D == 512 ? kEntryPm512 : kEntryPm128)
+         : plan->kernel == Kernel::kUmma ? kEntryUmma : kEntrySimt;
+    // One persistent CTA per SM, but no more than the work the call can have
+    // with every stream at max_len (the device splits the actual work).
+    const int64_t tiles_max = (int64_t)p.S * p.Hkv * head_work(p, st->max_len);
     int64_t grid = sms < kMaxCtas ? sms : kMaxCtas;
     if (tiles_max < grid)
         grid = tiles_max > 0 ? tiles_max : 1;
