@@ -39,16 +39,15 @@
 //              segment's end the sums are reduced across the block and the rows
 //              are normalised and stored, or left as partials for the merge.
 #include "launch.cuh"
-#include "plan.cuh"
-#include "umma.cuh"
+#include "ring.cuh"
 
 namespace tfp {
 
 namespace {
 
-constexpr int PT = 128;                  // key positions per tile (the MMA's M)
-constexpr uint32_t kBox = 16384;         // one [128 positions][64 dims] bf16 SW128 box
-constexpr uint32_t kUnit = 2 * kBox;     // one ring unit: 128 positions x 128 dims
+constexpr int PT = kRingTile;            // key positions per tile (the MMA's M)
+constexpr uint32_t kBox = kRingBox;      // one [128 positions][64 dims] bf16 SW128 box
+constexpr uint32_t kUnit = kRingUnit;    // one ring unit: 128 positions x 128 dims
 constexpr float kRescaleLog2 = 8.f;      // move a row's reference max only past this growth
 constexpr uint32_t kSmemCap = 232448;    // dynamic shared memory per block
 
@@ -118,36 +117,6 @@ struct PmArgs {
     CUtensorMap vmap;
 };
 
-template <class Sm>
-__device__ __forceinline__ bool pwait(Sm &sm, uint64_t *bar, uint32_t parity, uint32_t *flags,
-                                      uint32_t site)
-{
-    if (sm.abort_flag)
-        return false;
-    if (mbar_wait(bar, parity))
-        return true;
-    set_flag(flags, kDevTimeout);
-    set_flag(flags + 1, site);
-    sm.abort_flag = 1;
-    return false;
-}
-
-// OR of `pred` over the NT softmax threads (named barrier 1).
-template <int NT>
-__device__ __forceinline__ bool block_any(bool pred)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\t"
-        "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.or.pred po, 1, %2, pi;\n\t"
-        "selp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "n"(NT)
-        : "memory");
-    return r != 0;
-}
-
 // Reduces v[i] (one value per row, N rows) across the warp: lane l ends up
 // holding the reduction of rows [l * N / 32, (l + 1) * N / 32) in v[0 ..].
 // Each step sends half of the remaining rows to the partner lane.
@@ -183,76 +152,6 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, float (&x)[NR])
 #pragma unroll
         for (int e = 0; e < 32; ++e)
             x[32 * c + e] = __uint_as_float(r[e]);
-    }
-}
-
-// ---- producer ----------------------------------------------------------------
-
-// Loads the DB units of one K or V tile (positions [off, off + 128) of a page).
-template <int D, int NR>
-__device__ __forceinline__ bool pm_put_tile(const AttnParams &p, PmSmem<D, NR> &sm, uint32_t &U,
-                                            const CUtensorMap *map, int page, int kh, int off,
-                                            uint64_t pol)
-{
-    using C = PmCfg<D, NR>;
-    const bool page_ok = page >= 0 && page < p.n_pages;
-    if (!page_ok)
-        set_flag(p.flags, kDevBadPage);
-    const int y = ((page_ok ? page : 0) * p.Hkv + kh) * p.P + off;
-#pragma unroll 1
-    for (int kb = 0; kb < C::DB; ++kb) {
-        const int st = (int)(U % C::NU);
-        if (!pwait(sm, &sm.empty[st], ((U / C::NU) & 1u) ^ 1u, p.flags, kWaitEmpty))
-            return false;
-        if (page_ok) {
-            mbar_arrive_expect_tx(&sm.full[st], kUnit);
-            tma_load_2d(sm.ring[st], map, 128 * kb, y, &sm.full[st], pol);
-            tma_load_2d(sm.ring[st] + kBox, map, 128 * kb + 64, y, &sm.full[st], pol);
-        } else {
-            mbar_arrive(&sm.full[st]);
-        }
-        ++U;
-    }
-    return true;
-}
-
-// Unit order per segment (the issuer consumes in the same order):
-// K(0), then for each tile t: K(t + 1) if any, V(t).
-template <int D, int NR>
-__device__ __forceinline__ void pm_producer(const PmArgs &a, PmSmem<D, NR> &sm)
-{
-    using C = PmCfg<D, NR>;
-    const AttnParams &p = a.p;
-    const uint64_t pol = l2_evict_first_policy();
-    SegCursor cur;
-    cur.init(p, sm.range);
-    WorkItem it;
-    uint32_t U = 0;
-    bool ok = true;
-    while (ok && cur.next(p, it)) {
-        const int n = (it.key1 - it.key0 + PT - 1) / PT;
-        const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
-        int pg0 = __ldg(trow + it.key0 / p.P);
-        int pg1 = n > 1 ? __ldg(trow + (it.key0 + PT) / p.P) : 0;
-        ok = pm_put_tile(p, sm, U, &a.kmap, pg0, it.kh, it.key0 % p.P, pol);
-        for (int t = 0; ok && t < n; ++t) {
-            const int pos = it.key0 + t * PT;
-            const int pg2 = t + 2 < n ? __ldg(trow + (pos + 2 * PT) / p.P) : 0;
-            if (t + 1 < n)
-                ok = pm_put_tile(p, sm, U, &a.kmap, pg1, it.kh, (pos + PT) % p.P, pol);
-            if (ok)
-                ok = pm_put_tile(p, sm, U, &a.vmap, pg0, it.kh, pos % p.P, pol);
-            pg0 = pg1;
-            pg1 = pg2;
-        }
-    }
-    if (!ok || sm.abort_flag) {
-        // let the copies in flight land before the CTA exits
-        const uint32_t nf = U < (uint32_t)C::NU ? U : (uint32_t)C::NU;
-        for (uint32_t k = 1; k <= nf; ++k) {
-            const uint32_t v = U - k;
-            (void)mbar_wait(&sm.full[v % C::NU], (v / C::NU) & 1u);
-        }
     }
 }
 
@@ -557,7 +456,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
             const int nvalid = it.len - tpos;
             if (nvalid < PT) {
                 // the V units of this tile: K(0), then per tile K(t + 1) if any, V(t)
-                uint32_t uv = 2u * C::DB * u0 + C::DB * (2u * t + 1u + (t + 1 < n ? 1u : 0u));
+                uint32_t uv = ring_v_unit(C::DB, u0, t, n);
 #pragma unroll 1
                 for (int vb = 0; vb < C::DB; ++vb, ++uv) {
                     const int sl8 = (int)(uv % C::NU);
@@ -699,7 +598,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0)
-            pm_producer<D, NR>(a, sm);
+            ring_producer<PmCfg<D, NR>::DB, PmCfg<D, NR>::NU>(a.p, &a.kmap, &a.vmap, sm);
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0)

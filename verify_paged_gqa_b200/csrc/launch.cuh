@@ -28,11 +28,11 @@ cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream)
 template <int D>
 cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream);
 
-// Row-major tensor-core partial kernel (tcgen05): row blocks of
-// umma_rows(M) rows on the MMA's M.
-int umma_rows(int64_t M);
-bool umma_supported(const AttnParams &p);
-cudaError_t launch_attn_umma(const AttnParams &p, int grid, cudaStream_t stream);
+// Prompt tensor-core partial kernel (tcgen05): row blocks of prompt_rows()
+// rows on the QK MMA's M, PV transposed.
+int prompt_rows();
+bool prompt_supported(const AttnParams &p);
+cudaError_t launch_attn_prompt(const AttnParams &p, int grid, cudaStream_t stream);
 
 // Position-major tensor-core partial kernel: key positions on the MMA's M,
 // row blocks of pm_rows(p) rows (0: not supported for these arguments).

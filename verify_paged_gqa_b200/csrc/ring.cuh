@@ -1,0 +1,127 @@
+// ring.cuh -- the K/V ring shared by the two tensor-core partial kernels.
+//
+// A ring unit is 128 key positions x 128 head dims of one page x KV head
+// (K or V), loaded by TMA as two [128][64] bf16 boxes with 128-byte swizzle.
+// A tile of 128 positions at head dim D is DB = D / 128 units of K and DB of
+// V.  The producer loads, per segment, K(0) and then for each tile t the K
+// units of tile t + 1 (if any) followed by the V units of tile t: the MMA
+// issuer runs QK(t + 1) before PV(t), so it consumes the units in exactly
+// this order.  The kernel's shared-memory struct provides ring[NU][kRingUnit],
+// full[NU], empty[NU], range and abort_flag.
+#pragma once
+
+#include "plan.cuh"
+#include "umma.cuh"
+
+namespace tfp {
+
+constexpr int kRingTile = 128;             // positions per tile
+constexpr uint32_t kRingBox = 16384;       // one [128 positions][64 dims] bf16 box
+constexpr uint32_t kRingUnit = 2 * kRingBox;
+
+// mbarrier wait that records a timeout (status bit and wait site) and makes
+// every role of the CTA wind down.
+template <class Sm>
+__device__ __forceinline__ bool pwait(Sm &sm, uint64_t *bar, uint32_t parity, uint32_t *flags,
+                                      uint32_t site)
+{
+    if (sm.abort_flag)
+        return false;
+    if (mbar_wait(bar, parity))
+        return true;
+    set_flag(flags, kDevTimeout);
+    set_flag(flags + 1, site);
+    sm.abort_flag = 1;
+    return false;
+}
+
+// OR of `pred` over the NT threads of named barrier 1.
+template <int NT>
+__device__ __forceinline__ bool block_any(bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, %2, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "n"(NT)
+        : "memory");
+    return r != 0;
+}
+
+// Loads the DB units of one K or V tile (positions [off, off + 128) of a page).
+template <int DB, int NU, class Sm>
+__device__ __forceinline__ bool ring_put_tile(const AttnParams &p, Sm &sm, uint32_t &U,
+                                              const CUtensorMap *map, int page, int kh, int off,
+                                              uint64_t pol)
+{
+    const bool page_ok = page >= 0 && page < p.n_pages;
+    if (!page_ok)
+        set_flag(p.flags, kDevBadPage);
+    const int y = ((page_ok ? page : 0) * p.Hkv + kh) * p.P + off;
+#pragma unroll 1
+    for (int kb = 0; kb < DB; ++kb) {
+        const int st = (int)(U % NU);
+        if (!pwait(sm, &sm.empty[st], ((U / NU) & 1u) ^ 1u, p.flags, kWaitEmpty))
+            return false;
+        if (page_ok) {
+            mbar_arrive_expect_tx(&sm.full[st], kRingUnit);
+            tma_load_2d(sm.ring[st], map, 128 * kb, y, &sm.full[st], pol);
+            tma_load_2d(sm.ring[st] + kRingBox, map, 128 * kb + 64, y, &sm.full[st], pol);
+        } else {
+            mbar_arrive(&sm.full[st]);
+        }
+        ++U;
+    }
+    return true;
+}
+
+// One lane runs this.  Page ids are read two tiles ahead.
+template <int DB, int NU, class Sm>
+__device__ __forceinline__ void ring_producer(const AttnParams &p, const CUtensorMap *kmap,
+                                              const CUtensorMap *vmap, Sm &sm)
+{
+    constexpr int PT = kRingTile;
+    const uint64_t pol = l2_evict_first_policy();
+    SegCursor cur;
+    cur.init(p, sm.range);
+    WorkItem it;
+    uint32_t U = 0;
+    bool ok = true;
+    while (ok && cur.next(p, it)) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
+        int pg0 = __ldg(trow + it.key0 / p.P);
+        int pg1 = n > 1 ? __ldg(trow + (it.key0 + PT) / p.P) : 0;
+        ok = ring_put_tile<DB, NU>(p, sm, U, kmap, pg0, it.kh, it.key0 % p.P, pol);
+        for (int t = 0; ok && t < n; ++t) {
+            const int pos = it.key0 + t * PT;
+            const int pg2 = t + 2 < n ? __ldg(trow + (pos + 2 * PT) / p.P) : 0;
+            if (t + 1 < n)
+                ok = ring_put_tile<DB, NU>(p, sm, U, kmap, pg1, it.kh, (pos + PT) % p.P, pol);
+            if (ok)
+                ok = ring_put_tile<DB, NU>(p, sm, U, vmap, pg0, it.kh, pos % p.P, pol);
+            pg0 = pg1;
+            pg1 = pg2;
+        }
+    }
+    if (!ok || sm.abort_flag) {
+        // let the copies in flight land before the CTA exits
+        const uint32_t nf = U < (uint32_t)NU ? U : (uint32_t)NU;
+        for (uint32_t k = 1; k <= nf; ++k) {
+            const uint32_t v = U - k;
+            (void)mbar_wait(&sm.full[v % NU], (v / NU) & 1u);
+        }
+    }
+}
+
+// Ring index of the first V unit of tile t of a segment that starts at the
+// CTA's tile u0 and has n tiles (the order above).
+__device__ __forceinline__ uint32_t ring_v_unit(int DB, uint32_t u0, int t, int n)
+{
+    return 2u * DB * u0 + DB * (2u * t + 1u + (t + 1 < n ? 1u : 0u));
+}
+
+}  // namespace tfp

@@ -56,7 +56,7 @@ int check_pool_streams(const tf_kv_pool *pool, const tf_streams *st)
     return TF_OK;
 }
 
-enum class Kernel { kSimt, kUmma, kPm };
+enum class Kernel { kSimt, kPrompt, kPm };
 
 // Workspace: the 256-byte header (status word, wait site, the launch's tile
 // count at byte 64), each stream's first tile (int64), then two partial slots
@@ -74,7 +74,7 @@ size_t ws_part_offset(int S)
 // segment starts overlap with its deep ring and cost nothing measurable.
 constexpr int kEntryPm512 = 8;
 constexpr int kEntryPm128 = 4;
-constexpr int kEntryUmma = 4;
+constexpr int kEntryPrompt = 4;
 constexpr int kEntrySimt = 0;
 
 struct Plan {
@@ -127,9 +127,9 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
         if (nr > 0) {
             plan->kernel = Kernel::kPm;
             p.RB = nr;
-        } else if (umma_supported(p)) {
-            plan->kernel = Kernel::kUmma;
-            p.RB = umma_rows(M);
+        } else if (prompt_supported(p)) {
+            plan->kernel = Kernel::kPrompt;
+            p.RB = prompt_rows();
         }
     }
     p.n_rblk = static_cast<int32_t>((M + p.RB - 1) / p.RB);
@@ -138,7 +138,7 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     // Entry cost of a unit, in tiles: what starting one more unit costs a
     // CTA relative to streaming one tile of it (measured per kernel).
     p.VT = plan->kernel == Kernel::kPm ? (p.D == 512 ? kEntryPm512 : kEntryPm128)
-         : plan->kernel == Kernel::kUmma ? kEntryUmma : kEntrySimt;
+         : plan->kernel == Kernel::kPrompt ? kEntryPrompt : kEntrySimt;
     // One persistent CTA per SM, but no more than the work the call can have
     // with every stream at max_len (the device splits the actual work).
     const int64_t tiles_max = (int64_t)p.S * p.Hkv * head_work(p, st->max_len);
@@ -186,8 +186,8 @@ int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32
         e = launch_attn_pm(p, plan.grid, s);
         if (e == cudaSuccess)
             e = p.D == 128 ? launch_attn_merge<128>(p, s) : launch_attn_merge<512>(p, s);
-    } else if (plan.kernel == Kernel::kUmma) {
-        e = launch_attn_umma(p, plan.grid, s);
+    } else if (plan.kernel == Kernel::kPrompt) {
+        e = launch_attn_prompt(p, plan.grid, s);
         if (e == cudaSuccess)
             e = launch_attn_merge<128>(p, s);
     } else if (p.D == 128) {
