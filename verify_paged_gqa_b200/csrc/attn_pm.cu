@@ -455,6 +455,13 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
             // --- V rows past the stream's end: zero them (0 * NaN = NaN) ----
             const int nvalid = it.len - tpos;
             if (nvalid < PT) {
+                // The ring slots of this tile's V units last held units of
+                // V(t - 1) or earlier (at head dim 512 the ring is shorter than
+                // a tile): wait for PV(u - 1) first, so each full-barrier wait
+                // below names its own phase, not the one before it.
+                if (u >= 1)
+                    ok = pwait(sm, &sm.o_done[(u - 1) & 1u], ((u - 1) >> 1) & 1u, p.flags,
+                               kWaitEmpty) && ok;
                 // the V units of this tile: K(0), then per tile K(t + 1) if any, V(t)
                 uint32_t uv = ring_v_unit(C::DB, u0, t, n);
 #pragma unroll 1
