@@ -215,3 +215,13 @@ def test_split_skips_out_of_range_stream():
     ref = oracle.attend(case.q[keep], [case.k_lin[i] for i in keep], [case.v_lin[i] for i in keep],
                         case.lens[keep], 4, w.group, w.scale, threads=8)
     assert max_abs(out[keep], ref) <= TOL
+
+
+def test_split_prompt_kernel_more_units_than_ctas():
+    """Prompt rows on more (stream, KV head, row block) units than there are
+    CTAs: the prompt kernel runs the work split with partials and the merge
+    (with fewer units it takes one unit per CTA whole)."""
+    rng = np.random.default_rng(9400)
+    lens = [int(x) for x in rng.integers(64, 900, size=40)]
+    w = small_workload(128, 4, 512, 64, Hkv=2, seed=9401)
+    run_parity(w, lens, 64)

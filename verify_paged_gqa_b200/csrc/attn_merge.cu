@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
         }
         return;
     }
+    if (p.whole)
+        return;  // every unit was finished whole by one CTA
     // the unit's tiles [U0, U1) and the CTAs that met them: warp 0 works them
     // out once for the block (lanes split the row blocks)
     __shared__ int nseg_sh;

@@ -51,6 +51,7 @@ struct AttnParams {
     int32_t SR;                 // rows per partial slot: min(RB, M)
     int32_t n_cta;              // persistent CTAs of the partial kernel (the work split)
     int32_t VT;                 // entry tiles of work in front of every unit
+    int32_t whole;              // 1: CTA c takes unit c whole (no split, no partials)
     long long *first_tile;      // workspace: where each stream's work starts in the launch
     long long *total_tiles;     // workspace: work tiles of the launch
     float scale_log2;           // scale * log2(e): scores are kept in log2 units

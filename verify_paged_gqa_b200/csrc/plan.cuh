@@ -20,7 +20,9 @@
 // CTA's two workspace slots: slot 2c for a segment that starts at the CTA's
 // first tile, 2c + 1 for one that ends at its last (a CTA range meets at most
 // two units partially).  The merge kernel finds a split unit's segments from
-// the same arithmetic and combines them in position order.  A unit's result
+// the same arithmetic and combines them in position order.  (When the call
+// has no more units than CTAs, the tensor-bound prompt kernel instead gives
+// CTA c unit c whole: no partials and no merge.)  A unit's result
 // therefore depends on the lengths of the call's streams and the grid size
 // (never on the page table, nor on run-to-run timing).
 #pragma once
@@ -98,6 +100,31 @@ struct CtaRange {
 // workspace for the merge kernel.
 __device__ __forceinline__ void find_range(const AttnParams &p, CtaRange &out, int lane)
 {
+    if (p.whole) {
+        // CTA c takes unit c (stream, KV head, row block) whole
+        const int per_s = p.Hkv * p.n_rblk;
+        const int c = blockIdx.x;
+        const int s = c / per_s;
+        const int len = s < p.S ? __ldg(p.lens + s) : 0;
+        const long long hw = s < p.S ? head_work(p, len) : 0;
+        if (lane == 0) {
+            out.g0 = 0;
+            out.g1 = 0;
+            out.off0 = 0;
+            out.s0 = p.S;
+            if (hw > 0) {
+                const int kh = (c - s * per_s) / p.n_rblk;
+                const int b = c - s * per_s - kh * p.n_rblk;
+                long long before = 0;
+                for (int bb = 0; bb < b; ++bb)
+                    before += unit_work(p, len, bb);
+                out.s0 = s;
+                out.off0 = kh * hw + before;
+                out.g1 = unit_work(p, len, b);
+            }
+        }
+        return;
+    }
     long long tot = 0;
     for (int s = lane; s < p.S; s += 32)
         tot += p.Hkv * head_work(p, __ldg(p.lens + s));

@@ -145,6 +145,14 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     int64_t grid = sms < kMaxCtas ? sms : kMaxCtas;
     if (tiles_max < grid)
         grid = tiles_max > 0 ? tiles_max : 1;
+    // A tensor-bound prompt call with no more units than CTAs gives each CTA
+    // one whole unit: the split's partials and merge cost more than the
+    // idle SMs (measured on the chunked prompt).
+    const int64_t units = (int64_t)p.S * p.Hkv * p.n_rblk;
+    const int cap = sms < kMaxCtas ? sms : kMaxCtas;
+    p.whole = plan->kernel == Kernel::kPrompt && units <= cap ? 1 : 0;
+    if (p.whole)
+        grid = units > 0 ? units : 1;
     plan->grid = static_cast<int>(grid);
     p.n_cta = plan->grid;
     plan->ws_bytes = ws_part_offset(p.S) + (size_t)2 * plan->grid * p.SR * (p.D + 2) * sizeof(float);
