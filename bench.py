@@ -28,7 +28,10 @@ weak scaling, value = all ranks' bytes / the slowest rank's time.
 
 The default run also times the draft-verify workload (4 streams at 131,072
 positions, 4 KV / 32 query heads, 8-row windows) the same way and reports its
-verify tokens/s (window rows per second) under "verify" (--no-verify skips).
+verify tokens/s (window rows per second) under "verify", and likewise the head
+dim 512 verify workload ("hd512"), the 9,216-token chunked prompt ("prompt",
+causal TFLOP/s) and the shape variants ("variants": GQA 12, GQA 16 at head dim
+512, head dim 256); --no-verify skips them all.
 """
 from __future__ import annotations
 
@@ -580,6 +583,12 @@ def main():
         for name, key in (("verify_4x131k", "verify"), ("hd512_verify", "hd512"),
                           ("prompt_9216", "prompt")):
             line[key] = measure_other(name, args, barrier, dist, world, local)
+            torch.cuda.empty_cache()
+        # the shape variants the pages mention (GQA 12, GQA 16 at head dim 512,
+        # head dim 256), each timed the same way
+        line["variants"] = []
+        for name in ("gqa12_verify", "gqa16_hd512_decode", "hd256_verify"):
+            line["variants"].append(measure_other(name, args, barrier, dist, world, local))
             torch.cuda.empty_cache()
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

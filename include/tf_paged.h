@@ -89,7 +89,8 @@ extern "C" {
 #define TF_DEV_TIMEOUT 4u   /* a pipeline wait gave up (an internal error) */
 
 /* The pool: K and V pages, device memory, 16-byte aligned.
- * page_size must be a multiple of 64; head_dim must be 128 or 512. */
+ * page_size must be a multiple of 64; head_dim must be 128, 256 or 512
+ * (head dim 256 also needs page_size a multiple of 128). */
 typedef struct tf_kv_pool {
     void *k_pool;
     void *v_pool;

@@ -132,6 +132,13 @@ WORKLOADS = {
                              len_range=(2048, 9216)),
     "prompt_9216": Workload("prompt_9216", 1, 8, 4, 128, 512, 512, seed=5, lens=(9216,),
                             prompt_len=9216),
+    # shape variants the pages mention: GQA 12 (48 query / 4 KV heads), GQA 16
+    # at head dim 512 (16 query / 1 KV head), head dim 256
+    "gqa12_verify": Workload("gqa12_verify", 4, 4, 12, 128, 512, 8, seed=8, lens=(32768,) * 4),
+    "gqa16_hd512_decode": Workload("gqa16_hd512_decode", 16, 1, 16, 512, 512, 1, seed=9,
+                                   lens=(16384,) * 16),
+    "hd256_verify": Workload("hd256_verify", 16, 2, 8, 256, 512, 4, seed=10,
+                             len_range=(2048, 9216)),
     # smaller copies of the decode and verify workloads for profiler captures
     # (still larger than the 126 MB L2)
     "decode_12x8k": Workload("decode_12x8k", 12, 8, 4, 128, 512, 1, seed=6, lens=(8192,) * 12),

@@ -34,7 +34,7 @@ def test_parity_small_workload():
     run_parity(w, None, 1)
 
 
-@pytest.mark.parametrize("d", [128, 512])
+@pytest.mark.parametrize("d", [128, 256, 512])
 @pytest.mark.parametrize("G", [4, 8])
 @pytest.mark.parametrize("W", [1, 2, 3, 4, 8])
 def test_parity_sweep_page512(d, G, W):
@@ -152,7 +152,7 @@ def test_workspace_too_small_is_refused():
 
 
 @pytest.mark.parametrize("d,G,W", [(128, 8, 8), (128, 4, 3), (512, 8, 4), (512, 4, 8),
-                                   (128, 4, 1), (128, 4, 100)])
+                                   (256, 8, 4), (128, 4, 1), (128, 4, 100)])
 def test_parity_growing_scores(d, G, W):
     """K rows scaled up along the context: every row's max keeps growing past
     the kernels' rescale margin, so running maxima move and O is rescaled
@@ -225,3 +225,29 @@ def test_split_prompt_kernel_more_units_than_ctas():
     lens = [int(x) for x in rng.integers(64, 900, size=40)]
     w = small_workload(128, 4, 512, 64, Hkv=2, seed=9401)
     run_parity(w, lens, 64)
+
+
+# --- shape variants the pages mention: GQA 12 (48 query / 4 KV heads), GQA 16
+# at head dim 512 (16 query / 1 KV head), head dim 256
+
+@pytest.mark.parametrize("W", [1, 4, 8])
+def test_parity_gqa12(W):
+    w = synth.Workload("gqa12", 0, 4, 12, 128, 512, W, seed=9500 + W)
+    run_parity(w, [3000, 1025, W + 3], W)
+
+
+@pytest.mark.parametrize("W", [1, 4, 8])
+def test_parity_gqa16_hd512(W):
+    w = synth.Workload("gqa16", 0, 1, 16, 512, 512, W, seed=9600 + W)
+    run_parity(w, [5000, 700, W], W)
+
+
+def test_hd256_needs_pages_of_128():
+    import verify_paged_gqa_b200 as tf
+    w = small_workload(256, 4, 64, 1, seed=9700)
+    case = synth.make_case(w, lens=[300])
+    dc = DeviceCase(case)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tf.TFError) as e:
+        dc.attend(ws=ws)
+    assert e.value.status == tf.TF_EUNSUPPORTED

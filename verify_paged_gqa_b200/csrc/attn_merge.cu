@@ -186,6 +186,7 @@ cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream)
 }
 
 template cudaError_t launch_attn_merge<128>(const AttnParams &, cudaStream_t);
+template cudaError_t launch_attn_merge<256>(const AttnParams &, cudaStream_t);
 template cudaError_t launch_attn_merge<512>(const AttnParams &, cudaStream_t);
 
 }  // namespace tfp

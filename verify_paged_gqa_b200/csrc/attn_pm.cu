@@ -1,7 +1,7 @@
 // attn_pm.cu -- split-context paged attention on the 5th-generation tensor
 // cores with the key positions on the MMA's M dimension ("position-major"),
 // for row blocks of up to 64 query rows: draft-verify windows, decode at
-// GQA 8, and every head dim 512 case.
+// GQA 8, and every head dim 256 or 512 call.
 //
 // TensorFold #1620 ("Kolibri-1's full layers take their K/V from pages of
 // the core pool"), opening comment, "Reads": decode, verify and prompt rows
@@ -109,6 +109,7 @@ constexpr size_t pm_smem_bytes()
 
 static_assert(pm_smem_bytes<128, 32>() <= kSmemCap, "smem");
 static_assert(pm_smem_bytes<128, 64>() <= kSmemCap, "smem");
+static_assert(pm_smem_bytes<256, 32>() <= kSmemCap, "smem");
 static_assert(pm_smem_bytes<512, 32>() <= kSmemCap, "smem");
 
 struct PmArgs {
@@ -661,7 +662,7 @@ int pm_rows(const AttnParams &p)
         return 0;
     if (p.D == 128)
         return p.M <= 32 ? 32 : p.M <= 64 ? 64 : 0;
-    if (p.D == 512)
+    if (p.D == 256 || p.D == 512)
         return 32;
     return 0;
 }
@@ -672,6 +673,8 @@ cudaError_t launch_attn_pm(const AttnParams &p, int grid, cudaStream_t stream)
         return launch_pm<128, 32>(p, grid, stream);
     if (p.D == 128 && p.RB == 64)
         return launch_pm<128, 64>(p, grid, stream);
+    if (p.D == 256 && p.RB == 32)
+        return launch_pm<256, 32>(p, grid, stream);
     if (p.D == 512 && p.RB == 32)
         return launch_pm<512, 32>(p, grid, stream);
     return cudaErrorInvalidValue;

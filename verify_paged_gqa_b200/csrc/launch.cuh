@@ -26,7 +26,7 @@ size_t simt_smem_bytes();
 template <int D>
 cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream);
 template <int D>
-cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream);
+cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream);  // D 128, 256, 512
 
 // Prompt tensor-core partial kernel (tcgen05): row blocks of prompt_rows()
 // rows on the QK MMA's M, PV transposed.

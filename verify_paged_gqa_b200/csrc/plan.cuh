@@ -20,9 +20,9 @@
 // CTA's two workspace slots: slot 2c for a segment that starts at the CTA's
 // first tile, 2c + 1 for one that ends at its last (a CTA range meets at most
 // two units partially).  The merge kernel finds a split unit's segments from
-// the same arithmetic and combines them in position order.  (When the call
-// has no more units than CTAs, the tensor-bound prompt kernel instead gives
-// CTA c unit c whole: no partials and no merge.)  A unit's result
+// the same arithmetic and combines them in position order.  (When the call's
+// units fill most CTAs but not more, the tensor-bound prompt kernel instead
+// gives CTA c unit c whole: no partials and no merge.)  A unit's result
 // therefore depends on the lengths of the call's streams and the grid size
 // (never on the page table, nor on run-to-run timing).
 #pragma once

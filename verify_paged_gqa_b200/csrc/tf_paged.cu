@@ -39,7 +39,7 @@ int check_pool_streams(const tf_kv_pool *pool, const tf_streams *st)
         return TF_EINVAL;
     if (pool->n_pages < 1 || pool->n_kv_heads < 1 || pool->page_size < 1)
         return TF_EINVAL;
-    if (pool->head_dim != 128 && pool->head_dim != 512)
+    if (pool->head_dim != 128 && pool->head_dim != 256 && pool->head_dim != 512)
         return TF_EUNSUPPORTED;
     if (pool->page_size % 64 != 0)
         return TF_EUNSUPPORTED;
@@ -122,7 +122,14 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     // blocks with the rows there.
     plan->kernel = Kernel::kSimt;
     p.RB = kSimtRows;
-    if (M > kSimtRows) {
+    if (p.D == 256) {
+        // head dim 256 runs on the position-major kernel only (any row count)
+        const int nr = pm_rows(p);
+        if (nr == 0)
+            return TF_EUNSUPPORTED;
+        plan->kernel = Kernel::kPm;
+        p.RB = nr;
+    } else if (M > kSimtRows) {
         const int nr = pm_rows(p);
         if (nr > 0) {
             plan->kernel = Kernel::kPm;
@@ -145,12 +152,12 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     int64_t grid = sms < kMaxCtas ? sms : kMaxCtas;
     if (tiles_max < grid)
         grid = tiles_max > 0 ? tiles_max : 1;
-    // A tensor-bound prompt call with no more units than CTAs gives each CTA
-    // one whole unit: the split's partials and merge cost more than the
-    // idle SMs (measured on the chunked prompt).
+    // A tensor-bound prompt call whose units fill most CTAs (but no more)
+    // gives each CTA one whole unit: the split's partials and merge cost more
+    // than a few idle SMs (measured on the chunked prompt: 128 units on 148).
     const int64_t units = (int64_t)p.S * p.Hkv * p.n_rblk;
     const int cap = sms < kMaxCtas ? sms : kMaxCtas;
-    p.whole = plan->kernel == Kernel::kPrompt && units <= cap ? 1 : 0;
+    p.whole = plan->kernel == Kernel::kPrompt && units <= cap && 4 * units >= 3 * (int64_t)cap;
     if (p.whole)
         grid = units > 0 ? units : 1;
     plan->grid = static_cast<int>(grid);
@@ -193,7 +200,9 @@ int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32
     if (plan.kernel == Kernel::kPm) {
         e = launch_attn_pm(p, plan.grid, s);
         if (e == cudaSuccess)
-            e = p.D == 128 ? launch_attn_merge<128>(p, s) : launch_attn_merge<512>(p, s);
+            e = p.D == 128   ? launch_attn_merge<128>(p, s)
+                : p.D == 256 ? launch_attn_merge<256>(p, s)
+                             : launch_attn_merge<512>(p, s);
     } else if (plan.kernel == Kernel::kPrompt) {
         e = launch_attn_prompt(p, plan.grid, s);
         if (e == cudaSuccess)
