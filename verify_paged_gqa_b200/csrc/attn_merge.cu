@@ -11,10 +11,12 @@
 // in segment (position) order, so the result is the same on every run.
 //
 // The segments of a unit split across CTAs are found from the work split
-// (plan.cuh): the CTAs whose ranges meet the unit's real tiles, in order.  One block per (stream, KV head, row block, group of up to 8 rows);
-// one warp per row.  The weighted sum loads several segments' rows before
-// using them, so the loads of a round overlap.  Streams whose length is out
-// of range get NaN rows (and the status bit).
+// (plan.cuh): the CTAs whose ranges meet the unit's real tiles, in order.
+// One block per (stream, KV head, row block, group of up to 8 rows); one
+// warp per row.  A row's first round of O loads and its (m, l) loads are all
+// in flight together.  The kernel is launched as a programmatic dependent of
+// the partial kernel, so its launch overlaps that kernel's last CTAs.
+// Streams whose length is out of range get NaN rows (and the status bit).
 #include "launch.cuh"
 #include "plan.cuh"
 
@@ -46,6 +48,9 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
     if (m0 >= m1)
         return;
     const float NEG_INF = -__int_as_float(0x7f800000);
+    // launched as a programmatic dependent of the partial kernel: wait for
+    // that grid to complete (and its writes to be visible) before going on
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (!len_ok(p, len)) {
         if (threadIdx.x == 0 && kh == 0 && b == 0 && g == 0)
@@ -104,8 +109,35 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
 
     for (int m = m0 + warp; m < m1; m += nwarps) {
         const int r = m - mb;
-        float mx = NEG_INF;
-        for (int k = lane; k < nseg; k += 32) {
+        // The first round's O rows and the (m, l) of segments 0 .. 31 are
+        // loaded before any of them is used, so that one memory round trip
+        // covers a row with up to UK segments.
+        float w[UK];
+        float4 v[UK][NV];
+#pragma unroll
+        for (int kk = 0; kk < UK; ++kk) {
+            const int sl = kk < nseg ? slots[kk] : -1;
+#pragma unroll
+            for (int q = 0; q < NV; ++q)
+                v[kk][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (sl >= 0) {
+                const float *base = p.part + sl * slot_floats;
+#pragma unroll
+                for (int q = 0; q < NV; ++q)
+                    v[kk][q] = *reinterpret_cast<const float4 *>(base + (size_t)r * D + q * 128 +
+                                                                 lane * 4);
+            }
+        }
+        float m_lane = NEG_INF, l_lane = 0.f;  // segment k = lane
+        {
+            const int sl = lane < nseg ? slots[lane] : -1;
+            if (sl >= 0) {
+                m_lane = p.part[sl * slot_floats + (size_t)p.SR * D + r];
+                l_lane = p.part[sl * slot_floats + (size_t)p.SR * D + p.SR + r];
+            }
+        }
+        float mx = m_lane;
+        for (int k = lane + 32; k < nseg; k += 32) {
             const int sl = slots[k];
             if (sl >= 0)
                 mx = fmaxf(mx, p.part[sl * slot_floats + (size_t)p.SR * D + r]);
@@ -113,8 +145,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
 #pragma unroll
         for (int k = 16; k >= 1; k >>= 1)
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, k));
-        float l = 0.f;
-        for (int k = lane; k < nseg; k += 32) {
+        float l = (m_lane == NEG_INF) ? 0.f : l_lane * fast_exp2(m_lane - mx);
+        for (int k = lane + 32; k < nseg; k += 32) {
             const int sl = slots[k];
             if (sl < 0)
                 continue;
@@ -131,24 +163,31 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
         for (int e = 0; e < DL; ++e)
             acc[e] = 0.f;
         for (int k0 = 0; k0 < nseg; k0 += UK) {
-            float w[UK];
-            float4 v[UK][NV];
+            if (k0 > 0) {
 #pragma unroll
-            for (int kk = 0; kk < UK; ++kk) {
-                const int sl = k0 + kk < nseg ? slots[k0 + kk] : -1;
-                w[kk] = 0.f;
-#pragma unroll
-                for (int q = 0; q < NV; ++q)
-                    v[kk][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (sl >= 0) {
-                    const float *base = p.part + sl * slot_floats;
-                    const float mc = base[(size_t)p.SR * D + r];
-                    w[kk] = (mc == NEG_INF) ? 0.f : fast_exp2(mc - mx);
+                for (int kk = 0; kk < UK; ++kk) {
+                    const int sl = k0 + kk < nseg ? slots[k0 + kk] : -1;
 #pragma unroll
                     for (int q = 0; q < NV; ++q)
-                        v[kk][q] = *reinterpret_cast<const float4 *>(base + (size_t)r * D + q * 128 +
-                                                                     lane * 4);
+                        v[kk][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (sl >= 0) {
+                        const float *base = p.part + sl * slot_floats;
+#pragma unroll
+                        for (int q = 0; q < NV; ++q)
+                            v[kk][q] = *reinterpret_cast<const float4 *>(
+                                base + (size_t)r * D + q * 128 + lane * 4);
+                    }
                 }
+            }
+            // the weights, from the (m, l) loads above where the segment has a lane
+#pragma unroll
+            for (int kk = 0; kk < UK; ++kk) {
+                const int k = k0 + kk;
+                const int sl = k < nseg ? slots[k] : -1;
+                float mc = __shfl_sync(0xffffffffu, m_lane, k & 31);
+                if (k >= 32 && sl >= 0)
+                    mc = p.part[sl * slot_floats + (size_t)p.SR * D + r];
+                w[kk] = (sl < 0 || mc == NEG_INF) ? 0.f : fast_exp2(mc - mx);
             }
 #pragma unroll
             for (int kk = 0; kk < UK; ++kk) {
@@ -181,8 +220,19 @@ cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream)
     if (blocks == 0)
         return cudaSuccess;
     const int threads = 32 * min(kMergeRows, p.RB);
-    attn_merge_kernel<D><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(p);
-    return cudaGetLastError();
+    // programmatic dependent launch: the blocks are scheduled while the
+    // partial kernel runs out and wait for it in the kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attn_merge_kernel<D>, p);
 }
 
 template cudaError_t launch_attn_merge<128>(const AttnParams &, cudaStream_t);

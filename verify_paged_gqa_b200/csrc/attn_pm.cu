@@ -574,6 +574,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     PmSmem<D, NR> &sm = *reinterpret_cast<PmSmem<D, NR> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    allow_dependent_launch();
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {

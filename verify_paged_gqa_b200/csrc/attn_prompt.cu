@@ -423,6 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
     extern __shared__ uint8_t smem_raw[];
     PrSmem &sm = *reinterpret_cast<PrSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    allow_dependent_launch();
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {

@@ -609,6 +609,7 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     SimtSmem<D> &sm = *reinterpret_cast<SimtSmem<D> *>(smem_raw);
+    allow_dependent_launch();
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {

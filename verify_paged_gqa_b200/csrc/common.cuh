@@ -167,6 +167,13 @@ __device__ __forceinline__ void named_barrier(int id, int threads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Lets the next kernel in the stream, if it was launched as a programmatic
+// dependent (the merge), be scheduled now; it waits for this grid itself.
+__device__ __forceinline__ void allow_dependent_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void set_flag(uint32_t *flags, uint32_t bit)
 {
     atomicOr(flags, bit);
