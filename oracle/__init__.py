@@ -17,6 +17,11 @@ Sources for what is computed:
   * TensorFold pull request #2730 (eight-row verify window), "What this
     changes" and the checklist: a window is the pending token plus drafts,
     and drafted output equals undrafted output (causal inside the window).
+  * TensorFold pull request #1620, opening comment, first bullet and Reads
+    bullet: the verify kernels are "tree attention" over key groups of one
+    page.  The pages give no mask; the reading is a per-row bitmask over the
+    window's rows (its ancestors in the draft tree and itself), with every
+    position before the window visible (``attend(..., tree=...)``).
 """
 from __future__ import annotations
 
@@ -59,6 +64,9 @@ def open_library(path: str):
     lib.tfo_attend_units.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, f64,
                                      p, i64, p, i32]
     lib.tfo_attend_units.restype = ctypes.c_int
+    lib.tfo_attend_units_tree.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, f64,
+                                          p, p, i64, p, i32]
+    lib.tfo_attend_units_tree.restype = ctypes.c_int
     lib.tfo_put_rows.argtypes = [p, p, i32, i32, i32, i32, p, i32, p, i32, p, p, i32]
     lib.tfo_put_rows.restype = ctypes.c_int
     return lib
@@ -89,7 +97,8 @@ def _pack_linear(caches):
     return flat, offs
 
 
-def attend(q, k_lin, v_lin, lens, rows, group, scale, units=None, threads=1, lib=None):
+def attend(q, k_lin, v_lin, lens, rows, group, scale, units=None, threads=1, lib=None,
+           tree=None):
     """Softmax attention over linear caches, in fp64.
 
     q      : uint16 (bf16 bits) [S][rows][Hq][d]
@@ -99,6 +108,9 @@ def attend(q, k_lin, v_lin, lens, rows, group, scale, units=None, threads=1, lib
     group  : query heads per KV head G (query head h reads KV head h // G)
     units  : optional int array [n][3] of (s, r, h); then returns [n][d]
     lib    : optional library from ``open_library`` (default: the built oracle)
+    tree   : optional uint8 [S][rows] row masks (rows <= 8): bit c of tree[s][r]
+             set means row r sees window row c; positions before the window
+             are seen by every row.  None is the causal window.
     Returns float64 [S][rows][Hq][d] (or [n][d] for ``units``).
     """
     lib = lib or _load()
@@ -118,9 +130,16 @@ def attend(q, k_lin, v_lin, lens, rows, group, scale, units=None, threads=1, lib
                                      indexing="ij"), axis=-1).reshape(-1, 3)
     units = np.ascontiguousarray(units, dtype=np.int32)
     out = np.zeros((units.shape[0], d), dtype=np.float64)
-    st = lib.tfo_attend_units(_ptr(q), _ptr(kf), _ptr(vf), _ptr(offs), _ptr(lens), S, W, Hkv,
-                              group, d, float(scale), _ptr(units), units.shape[0], _ptr(out),
-                              int(threads))
+    if tree is None:
+        st = lib.tfo_attend_units(_ptr(q), _ptr(kf), _ptr(vf), _ptr(offs), _ptr(lens), S, W,
+                                  Hkv, group, d, float(scale), _ptr(units), units.shape[0],
+                                  _ptr(out), int(threads))
+    else:
+        tree = np.ascontiguousarray(tree, dtype=np.uint8)
+        assert tree.shape == (S, W)
+        st = lib.tfo_attend_units_tree(_ptr(q), _ptr(kf), _ptr(vf), _ptr(offs), _ptr(lens), S,
+                                       W, Hkv, group, d, float(scale), _ptr(tree), _ptr(units),
+                                       units.shape[0], _ptr(out), int(threads))
     if st != 0:
         raise ValueError(f"oracle attend refused its arguments (status {st})")
     return out.reshape(S, W, Hq, d) if full else out

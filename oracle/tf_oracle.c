@@ -33,6 +33,17 @@
  *     x_j = scale * sum_i q[s][r][h][i] * K_s[j][kh][i]      j = 0..t
  *     o[s][r][h][i] = sum_j exp(x_j - max x) V_s[j][kh][i] / sum_j exp(x_j - max x)
  *
+ * Tree-mask verify (tfo_attend_units_tree).  The same page names the
+ * verify kernels "tree attention" and calls the 512-position pages its key
+ * groups (opening comment, first bullet and Reads bullet); it gives no mask.
+ * The reading used here: a window of W rows is a draft tree laid out in
+ * order, and row r carries a bitmask tree[s][r] over the window's rows --
+ * bit c set means row r sees window row c (its ancestors and itself).  Every
+ * position before the window is seen by every row.  So row r attends to
+ *     { j < len_s - W }  U  { len_s - W + c : bit c of tree[s][r] }
+ * and the causal window above is the chain mask tree[s][r] = 2^(r+1) - 1.
+ * A row whose set is empty is refused (status -1).
+ *
  * Everything is fp64; bf16 inputs are exact in fp64.  One unit (s, r, h)
  * is computed by one thread start to finish in a fixed order, so the result
  * does not depend on how many threads run.
@@ -63,6 +74,7 @@ typedef struct {
     const int32_t *lens;
     int32_t S, W, Hkv, G, d;
     double scale;
+    const uint8_t *tree;    /* NULL (causal), or [S][W] row masks */
     const int32_t *units;   /* n_units triples (s, r, h) */
     int64_t n_units;
     double *out;            /* [n_units][d] */
@@ -71,43 +83,62 @@ typedef struct {
     int32_t status;
 } attend_job;
 
-/* One output row, straight from the definition above. */
+/* Whether row r of stream s sees position j (the definitions above). */
+static int row_sees(const attend_job *J, int32_t s, int32_t r, int64_t j)
+{
+    const int64_t base = (int64_t)J->lens[s] - J->W;  /* the window's first position */
+    if (j < base)
+        return 1;
+    if (j >= J->lens[s])
+        return 0;
+    if (J->tree == NULL)
+        return j <= base + r;
+    return (J->tree[(int64_t)s * J->W + r] >> (j - base)) & 1;
+}
+
+/* One output row, straight from the definition above: the scores of the
+ * positions the row sees, in position order, then the softmax and the
+ * weighted sum of their values. */
 static int attend_one(const attend_job *J, int32_t s, int32_t r, int32_t h,
-                      double *o, double *x, double *w)
+                      double *o, double *x, double *w, int64_t *pos)
 {
     const int32_t Hq = J->Hkv * J->G;
     const int32_t d = J->d;
     const int32_t kh = h / J->G;
-    const int64_t t = (int64_t)J->lens[s] - J->W + r;
     const uint16_t *qrow = J->q + (((int64_t)s * J->W + r) * Hq + h) * d;
     const uint16_t *ks = J->k + J->kv_off[s];
     const uint16_t *vs = J->v + J->kv_off[s];
-    int64_t j;
+    int64_t j, n = 0;
     int32_t i;
     double mx, l;
 
-    if (t < 0)
+    if ((int64_t)J->lens[s] - J->W + r < 0)
         return -1;
-    for (j = 0; j <= t; ++j) {
-        const uint16_t *krow = ks + (j * J->Hkv + kh) * d;
+    for (j = 0; j < J->lens[s]; ++j)
+        if (row_sees(J, s, r, j))
+            pos[n++] = j;
+    if (n == 0)
+        return -1;
+    for (j = 0; j < n; ++j) {
+        const uint16_t *krow = ks + (pos[j] * J->Hkv + kh) * d;
         double acc = 0.0;
         for (i = 0; i < d; ++i)
             acc += bf16_to_double(qrow[i]) * bf16_to_double(krow[i]);
         x[j] = J->scale * acc;
     }
     mx = x[0];
-    for (j = 1; j <= t; ++j)
+    for (j = 1; j < n; ++j)
         if (x[j] > mx)
             mx = x[j];
     l = 0.0;
-    for (j = 0; j <= t; ++j) {
+    for (j = 0; j < n; ++j) {
         w[j] = exp(x[j] - mx);
         l += w[j];
     }
     for (i = 0; i < d; ++i)
         o[i] = 0.0;
-    for (j = 0; j <= t; ++j) {
-        const uint16_t *vrow = vs + (j * J->Hkv + kh) * d;
+    for (j = 0; j < n; ++j) {
+        const uint16_t *vrow = vs + (pos[j] * J->Hkv + kh) * d;
         for (i = 0; i < d; ++i)
             o[i] += w[j] * bf16_to_double(vrow[i]);
     }
@@ -122,40 +153,45 @@ static void *attend_worker(void *arg)
     int64_t maxlen = 1, u;
     int32_t s;
     double *x, *w;
+    int64_t *pos;
 
     for (s = 0; s < J->S; ++s)
         if (J->lens[s] > maxlen)
             maxlen = J->lens[s];
     x = (double *)malloc(sizeof(double) * (size_t)maxlen);
     w = (double *)malloc(sizeof(double) * (size_t)maxlen);
-    if (!x || !w) {
+    pos = (int64_t *)malloc(sizeof(int64_t) * (size_t)maxlen);
+    if (!x || !w || !pos) {
         J->status = -2;
         free(x);
         free(w);
+        free(pos);
         return NULL;
     }
     for (u = J->tid; u < J->n_units; u += J->nthreads) {
         const int32_t *t3 = J->units + 3 * u;
-        if (attend_one(J, t3[0], t3[1], t3[2], J->out + u * J->d, x, w) != 0) {
+        if (attend_one(J, t3[0], t3[1], t3[2], J->out + u * J->d, x, w, pos) != 0) {
             J->status = -1;
             break;
         }
     }
     free(x);
     free(w);
+    free(pos);
     return NULL;
 }
 
 /*
- * Attention for a list of (stream, window row, query head) units.
+ * Attention for a list of (stream, window row, query head) units, with the
+ * window's rows either causal (tree == NULL) or under per-row tree masks.
  * Returns 0, or -1 on a bad argument (a row before position 0, a unit out
- * of range), -2 when memory runs out.
+ * of range, a row that sees nothing), -2 when memory runs out.
  */
-int tfo_attend_units(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                     const int64_t *kv_off, const int32_t *lens, int32_t S,
-                     int32_t W, int32_t Hkv, int32_t G, int32_t d, double scale,
-                     const int32_t *units, int64_t n_units, double *out,
-                     int32_t nthreads)
+int tfo_attend_units_tree(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int64_t *kv_off, const int32_t *lens, int32_t S,
+                          int32_t W, int32_t Hkv, int32_t G, int32_t d, double scale,
+                          const uint8_t *tree, const int32_t *units, int64_t n_units,
+                          double *out, int32_t nthreads)
 {
     attend_job *jobs;
     pthread_t *th;
@@ -164,6 +200,8 @@ int tfo_attend_units(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 
     if (S <= 0 || W <= 0 || Hkv <= 0 || G <= 0 || d <= 0 || n_units < 0)
         return -1;
+    if (tree != NULL && W > 8)
+        return -1;  /* one mask byte per row */
     for (u = 0; u < n_units; ++u) {
         const int32_t *t3 = units + 3 * u;
         if (t3[0] < 0 || t3[0] >= S || t3[1] < 0 || t3[1] >= W || t3[2] < 0 ||
@@ -185,7 +223,7 @@ int tfo_attend_units(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         attend_job *J = &jobs[t];
         J->q = q; J->k = k; J->v = v; J->kv_off = kv_off; J->lens = lens;
         J->S = S; J->W = W; J->Hkv = Hkv; J->G = G; J->d = d; J->scale = scale;
-        J->units = units; J->n_units = n_units; J->out = out;
+        J->tree = tree; J->units = units; J->n_units = n_units; J->out = out;
         J->nthreads = nthreads; J->tid = t; J->status = 0;
     }
     if (nthreads == 1) {
@@ -207,6 +245,17 @@ int tfo_attend_units(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     free(jobs);
     free(th);
     return st;
+}
+
+/* The causal window: tfo_attend_units_tree without masks. */
+int tfo_attend_units(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     const int64_t *kv_off, const int32_t *lens, int32_t S,
+                     int32_t W, int32_t Hkv, int32_t G, int32_t d, double scale,
+                     const int32_t *units, int64_t n_units, double *out,
+                     int32_t nthreads)
+{
+    return tfo_attend_units_tree(q, k, v, kv_off, lens, S, W, Hkv, G, d, scale, NULL, units,
+                                 n_units, out, nthreads);
 }
 
 /*

@@ -27,7 +27,10 @@ Workloads (synthetic stand-ins for the pages' served runs):
     query heads, d 512, 4-row windows, K/V ~ N(0, 0.5^2) (TensorFold #1620's
     head dim 512 global layer, four-row cells);
   * ``prompt_9216``    one 9,216-token prompt written into shuffled pages, then
-    attended in causal chunks of 512 rows, 8 KV / 32 query heads, d 128.
+    attended in causal chunks of 512 rows, 8 KV / 32 query heads, d 128;
+  * ``tree_verify_4x131k`` the verify workload with every stream's window a
+    random draft tree (TensorFold #1620 calls the verify kernels "tree
+    attention"; each row sees its ancestors and itself).
 """
 from __future__ import annotations
 
@@ -111,6 +114,7 @@ class Workload:
     pool_factor: float = 1.2
     n_pages: int = 0           # fixed pool size (0: ceil(pool_factor * needed) + 1)
     prompt_len: int = 0        # >0: one prompt attended in chunks of ``rows``
+    tree: bool = False         # verify windows under random draft-tree masks
 
     @property
     def n_q_heads(self) -> int:
@@ -139,11 +143,43 @@ WORKLOADS = {
                                    lens=(16384,) * 16),
     "hd256_verify": Workload("hd256_verify", 16, 2, 8, 256, 512, 4, seed=10,
                              len_range=(2048, 9216)),
+    # the verify workload with each stream's 8 rows a random draft tree
+    "tree_verify_4x131k": Workload("tree_verify_4x131k", 4, 4, 8, 128, 512, 8, seed=11,
+                                   lens=(131072,) * 4, tree=True),
     # smaller copies of the decode and verify workloads for profiler captures
     # (still larger than the 126 MB L2)
     "decode_12x8k": Workload("decode_12x8k", 12, 8, 4, 128, 512, 1, seed=6, lens=(8192,) * 12),
     "verify_4x16k": Workload("verify_4x16k", 4, 4, 8, 128, 512, 8, seed=7, lens=(16384,) * 4),
 }
+
+
+def tree_masks(key, n_streams: int, rows: int) -> np.ndarray:
+    """Random draft trees, one per stream: row 0 is the root and row r > 0 hangs
+    under a parent drawn uniformly from rows 0 .. r - 1.  Returns uint8
+    [S][rows] with bit c of [s][r] set when window row c is row r or one of its
+    ancestors (the mask a tree-verify call takes)."""
+    assert 1 <= rows <= 8
+    rng = _rng(*key)
+    out = np.zeros((n_streams, rows), dtype=np.uint8)
+    for s in range(n_streams):
+        for r in range(rows):
+            parent_mask = int(out[s, int(rng.integers(0, r))]) if r > 0 else 0
+            out[s, r] = parent_mask | (1 << r)
+    return out
+
+
+def chain_masks(n_streams: int, rows: int) -> np.ndarray:
+    """The causal window as tree masks: row r sees rows 0 .. r."""
+    return np.tile(np.array([(1 << (r + 1)) - 1 for r in range(rows)], dtype=np.uint8),
+                   (n_streams, 1))
+
+
+def workload_tree(w: Workload, n_streams: int | None = None, rows: int | None = None):
+    """The tree masks of a tree workload (None for a causal one)."""
+    if not w.tree:
+        return None
+    return tree_masks((w.seed, 7), w.n_streams if n_streams is None else n_streams,
+                      w.rows if rows is None else rows)
 
 
 def stream_lens(w: Workload) -> np.ndarray:

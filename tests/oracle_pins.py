@@ -16,7 +16,11 @@ What pins what:
     key;
   * invariants: causality, verify row == decode at that position, thread
     count does not change a bit;
-  * the row write: per-element brute force on a tiny pool, untouched bytes.
+  * the row write: per-element brute force on a tiny pool, untouched bytes;
+  * tree masks: a hand-derived tree with siblings, brute force and torch's
+    attention with the explicit mask, every tree row equal (to the bit) to a
+    decode over the keys on its path, and chain masks equal to the causal
+    window.
 """
 from __future__ import annotations
 
@@ -55,12 +59,14 @@ def pin_hand_examples(lib=None):
         q = _bf(ex["q"])
         k = [_bf(x) for x in ex["k"]]
         v = [_bf(x) for x in ex["v"]]
-        out = oracle.attend(q, k, v, ex["lens"], ex["W"], ex["G"], scales[ex["scale"]], lib=lib)
+        tree = np.array(ex["tree"], dtype=np.uint8) if "tree" in ex else None
+        out = oracle.attend(q, k, v, ex["lens"], ex["W"], ex["G"], scales[ex["scale"]], lib=lib,
+                            tree=tree)
         np.testing.assert_allclose(out, np.array(ex["out"]), rtol=0, atol=1e-13,
                                    err_msg=ex["name"])
 
 
-def brute_force(q, k, v, lens, W, G, scale):
+def brute_force(q, k, v, lens, W, G, scale, tree=None):
     """Pure-Python attention: full score matrix, explicit mask, no max shift."""
     S, _, Hq, d = q.shape
     qf = _f64(q)
@@ -73,7 +79,10 @@ def brute_force(q, k, v, lens, W, G, scale):
                 g = h // G
                 e = []
                 for j in range(n):
-                    visible = j <= n - W + r
+                    if tree is None:
+                        visible = j <= n - W + r
+                    else:
+                        visible = j < n - W or (int(tree[s][r]) >> (j - (n - W))) & 1 == 1
                     if visible:
                         x = scale * math.fsum(qf[s, r, h, i] * kf[j, g, i] for i in range(d))
                         e.append((j, math.exp(x)))
@@ -211,5 +220,71 @@ def pin_put_rows(lib=None):
     np.testing.assert_array_equal(vp, want_v)
 
 
+def _tree_case(rng, S, W, Hkv, G, d, lens, key):
+    q, k, v = _random_case(rng, S, W, Hkv, G, d, lens)
+    return q, k, v, synth.tree_masks(key, S, W)
+
+
+def _visible(n, W, mask):
+    return [j for j in range(n) if j < n - W or (int(mask) >> (j - (n - W))) & 1]
+
+
+def pin_tree_brute_force(lib=None):
+    rng = np.random.default_rng(16)
+    for i, (S, W, Hkv, G, d, lens) in enumerate([(2, 4, 1, 2, 4, [5, 4]), (1, 8, 2, 1, 4, [11]),
+                                                  (3, 3, 1, 3, 3, [3, 7, 4])]):
+        q, k, v, tree = _tree_case(rng, S, W, Hkv, G, d, lens, (99, i))
+        scale = 1.0 / math.sqrt(d)
+        got = oracle.attend(q, k, v, lens, W, G, scale, lib=lib, tree=tree)
+        want = brute_force(q, k, v, lens, W, G, scale, tree=tree)
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+
+
+def pin_tree_sdpa(lib=None):
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(17)
+    for i, (S, W, Hkv, G, d, lens) in enumerate([(3, 8, 2, 4, 16, [8, 40, 19]),
+                                                  (2, 5, 1, 8, 32, [9, 70])]):
+        q, k, v, tree = _tree_case(rng, S, W, Hkv, G, d, lens, (98, i))
+        scale = 1.0 / math.sqrt(d)
+        got = oracle.attend(q, k, v, lens, W, G, scale, lib=lib, tree=tree)
+        for s in range(S):
+            n = lens[s]
+            qt = torch.from_numpy(_f64(q[s])).permute(1, 0, 2)[None]
+            kt = torch.from_numpy(_f64(k[s])).permute(1, 0, 2)[None]
+            vt = torch.from_numpy(_f64(v[s])).permute(1, 0, 2)[None]
+            mask = torch.zeros((W, n), dtype=torch.bool)
+            for r in range(W):
+                mask[r, _visible(n, W, tree[s][r])] = True
+            ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale,
+                                                 enable_gqa=True)
+            np.testing.assert_allclose(got[s], ref[0].permute(1, 0, 2).numpy(), rtol=0,
+                                       atol=1e-12)
+
+
+def pin_tree_paths(lib=None):
+    # a tree row attends exactly to the keys on its root path: the same as one
+    # decode row over a cache holding only those keys, in order (to the bit)
+    rng = np.random.default_rng(18)
+    S, W, Hkv, G, d = 3, 8, 2, 2, 8
+    lens = [8, 21, 13]
+    q, k, v, tree = _tree_case(rng, S, W, Hkv, G, d, lens, (97, 0))
+    scale = 0.3
+    got = oracle.attend(q, k, v, lens, W, G, scale, lib=lib, tree=tree)
+    for s in range(S):
+        for r in range(W):
+            vis = _visible(lens[s], W, tree[s][r])
+            out = oracle.attend(q[s:s + 1, r:r + 1].copy(), [k[s][vis]], [v[s][vis]], [len(vis)],
+                                1, G, scale, lib=lib)
+            np.testing.assert_array_equal(out[0, 0], got[s, r])
+    # chain masks are the causal window, to the bit
+    base = oracle.attend(q, k, v, lens, W, G, scale, lib=lib)
+    chain = oracle.attend(q, k, v, lens, W, G, scale, lib=lib, tree=synth.chain_masks(S, W))
+    np.testing.assert_array_equal(chain, base)
+    # and a tree with a branch differs from it
+    assert np.abs(got - base).max() > 1e-3
+
+
 ALL_PINS = [pin_hand_examples, pin_brute_force, pin_sdpa, pin_closed_forms, pin_invariants,
-            pin_put_rows]
+            pin_put_rows, pin_tree_brute_force, pin_tree_sdpa, pin_tree_paths]

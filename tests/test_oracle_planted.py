@@ -14,10 +14,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "tf_oracle.c")
 # buffers (no out-of-range positions), so a failing pin is an assertion, not a crash.
 PLANTS = [
     ("gqa mapping by modulo", "const int32_t kh = h / J->G;", "const int32_t kh = h % J->Hkv;"),
-    ("window one position early", "(int64_t)J->lens[s] - J->W + r;",
-     "(int64_t)J->lens[s] - J->W + r - 1;"),
-    ("window ignores row index", "(int64_t)J->lens[s] - J->W + r;",
-     "(int64_t)J->lens[s] - J->W;"),
+    ("window one position early", "return j <= base + r;", "return j <= base + r - 1;"),
+    ("window ignores row index", "return j <= base + r;", "return j <= base;"),
     ("softmax sign flipped", "w[j] = exp(x[j] - mx);", "w[j] = exp(mx - x[j]);"),
     ("scale dropped", "x[j] = J->scale * acc;", "x[j] = acc;"),
     ("no normalisation", "o[i] /= l;", "o[i] /= 1.0;"),
@@ -25,10 +23,16 @@ PLANTS = [
      "const uint16_t *vs = J->k + J->kv_off[s];"),
     ("query rows transposed", "(((int64_t)s * J->W + r) * Hq + h) * d;",
      "(((int64_t)s * Hq + h) * J->W + r) * d;"),
-    ("key cache read head-major", "const uint16_t *krow = ks + (j * J->Hkv + kh) * d;",
-     "const uint16_t *krow = ks + ((int64_t)kh * J->lens[s] + j) * d;"),
-    ("last key dropped from the sum", "for (j = 0; j <= t; ++j) {\n        w[j]",
-     "for (j = 0; j < t; ++j) {\n        w[j]"),
+    ("key cache read head-major", "const uint16_t *krow = ks + (pos[j] * J->Hkv + kh) * d;",
+     "const uint16_t *krow = ks + ((int64_t)kh * J->lens[s] + pos[j]) * d;"),
+    ("last key dropped from the sum", "for (j = 0; j < n; ++j) {\n        w[j]",
+     "for (j = 0; j < n - 1; ++j) {\n        w[j]"),
+    ("tree bit taken by row, not key", "return (J->tree[(int64_t)s * J->W + r] >> (j - base)) & 1;",
+     "return (J->tree[(int64_t)s * J->W + r] >> r) & 1;"),
+    ("tree mask of the mirrored row", "return (J->tree[(int64_t)s * J->W + r] >> (j - base)) & 1;",
+     "return (J->tree[(int64_t)s * J->W + (J->W - 1 - r)] >> (j - base)) & 1;"),
+    ("tree mask shifted by one key", "return (J->tree[(int64_t)s * J->W + r] >> (j - base)) & 1;",
+     "return (J->tree[(int64_t)s * J->W + r] >> (j - base + 1)) & 1;"),
     ("row write slot off by one", "const int64_t slot = pos % P;",
      "const int64_t slot = (pos + 1) % P;"),
     ("row write pool index transposed", "(((int64_t)page * Hkv + kh) * P + slot) * d;",
