@@ -262,8 +262,13 @@ class Workload:
             self.q = synth.q_rows_torch(w, S, W, device=device)     # [S][W][Hq][d]
             self.chunk_lens = None
             self.bytes_per_step = kv_bytes(self.lens_np, Hkv, d)
-            self.flops_per_step = 4 * d * Hq * sum(
-                int(n) - W + r + 1 for n in self.lens_np for r in range(W))
+            self.tree_np = synth.workload_tree(w)
+            if self.tree_np is None:
+                seen = [int(n) - W + r + 1 for n in self.lens_np for r in range(W)]
+            else:   # the positions before the window plus the window rows each mask names
+                seen = [int(n) - W + bin(int(self.tree_np[s, r]) & ((1 << W) - 1)).count("1")
+                        for s, n in enumerate(self.lens_np) for r in range(W)]
+            self.flops_per_step = 4 * d * Hq * sum(seen)
             self.rows_per_step = S * W
         self.out = torch.empty(self.q.shape, dtype=torch.float32, device=device)
         self.bytes_in_l2 = kv_bytes(self.lens_np, Hkv, d) < L2_BYTES
@@ -272,6 +277,10 @@ class Workload:
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         self.attn_fn = (tf.tf_paged_attn_decode if W == 1 else
                         tf.tf_paged_attn_verify if W <= 8 else tf.tf_paged_attn_prompt)
+        if not w.prompt_len and self.tree_np is not None:
+            self.tree = torch.from_numpy(self.tree_np).to(device)
+            self.attn_fn = lambda kp, vp, tb, ln, q, sc, out, ws, ml: tf.tf_paged_attn_verify_tree(
+                kp, vp, tb, ln, q, self.tree, sc, out, ws, ml)
         torch.cuda.synchronize()
 
     def parts(self, k_new=None, v_new=None, q=None):
@@ -503,6 +512,8 @@ def workload_config(name):
            "kv_heads": w.n_kv_heads, "q_heads": w.n_q_heads, "head_dim": w.head_dim,
            "page_size": w.page_size, "rows": w.rows, "parallelism": "replicas",
            "l2": f"inputs {kv_bytes(lens, w.n_kv_heads, w.head_dim) / 1e9:.2f} GB > 126 MB L2"}
+    if w.tree:
+        cfg["window"] = "seeded random draft tree per stream (row r sees its ancestors and itself)"
     if w.prompt_len:
         cfg["chunks"] = w.prompt_len // w.rows
         cfg["l2"] = (f"K/V {kv_bytes(lens, w.n_kv_heads, w.head_dim) / 1e6:.1f} MB < 126 MB L2: "
@@ -587,7 +598,7 @@ def main():
         # the shape variants the pages mention (GQA 12, GQA 16 at head dim 512,
         # head dim 256), each timed the same way
         line["variants"] = []
-        for name in ("gqa12_verify", "gqa16_hd512_decode", "hd256_verify"):
+        for name in ("gqa12_verify", "gqa16_hd512_decode", "hd256_verify", "tree_verify_4x131k"):
             line["variants"].append(measure_other(name, args, barrier, dist, world, local))
             torch.cuda.empty_cache()
 

@@ -120,7 +120,8 @@ TF_API int tf_kv_put_rows(const tf_kv_pool *pool, const tf_streams *streams,
                    void *stream);
 
 /* Workspace bytes an attention call with these arguments needs on the
- * current device (0 on a bad argument).  The workspace holds split-context
+ * current device (0 on a bad argument), for any of the attention calls
+ * with these arguments (tf_paged_attn_verify_tree included).  The workspace holds split-context
  * partial results and, in its first 4 bytes, the device status word, which
  * the calls only OR bits into: zero those 4 bytes once after allocating
  * (cudaMemset, or one tf_workspace_status call).  The rest needs no
@@ -144,6 +145,29 @@ TF_API int tf_paged_attn_verify(const tf_kv_pool *pool, const tf_streams *stream
                          const void *q, int32_t n_q_heads, int32_t rows,
                          float scale, float *out, void *workspace,
                          size_t workspace_bytes, void *stream);
+
+/* Draft-verify window whose rows form a draft tree (TensorFold #1620,
+ * opening comment, first and Reads bullets: drafted verify runs through
+ * "tree attention" kernels whose key groups are the 512-position pages; the
+ * pages give no mask, so this reading: a window of `rows` drafted tokens,
+ * laid out in order, each seeing the positions before the window and the
+ * window rows named by its mask).
+ *  tree_masks  device, uint8 [n_streams][rows], caller-owned, read during the
+ *              call: bit c of tree_masks[s][r] set means row r of stream s
+ *              sees window row c (position lens[s] - rows + c).  A draft tree
+ *              gives row r its ancestors and itself; the causal window of
+ *              tf_paged_attn_verify is the chain mask 2^(r+1) - 1.  Bits at or
+ *              above `rows` are ignored.  A row that sees no position at all
+ *              (no context before the window and an empty mask) gets NaN.
+ * Everything else (arguments, layouts, results, the workspace, errors) is
+ * as tf_paged_attn_verify; TF_EINVAL also when tree_masks is null, and
+ * TF_EUNSUPPORTED when page_size is not a multiple of 128.  Head dim 128
+ * calls with more than 64 query rows per KV head (G * rows) read each K/V
+ * tile once per 64 rows. */
+TF_API int tf_paged_attn_verify_tree(const tf_kv_pool *pool, const tf_streams *streams,
+                              const void *q, int32_t n_q_heads, int32_t rows,
+                              const uint8_t *tree_masks, float scale, float *out,
+                              void *workspace, size_t workspace_bytes, void *stream);
 
 /* Chunked prompt rows (TensorFold #1620 "Reads": prompts through the paged
  * prompt kernels).  The same causal rule as verify for a chunk of

@@ -51,13 +51,18 @@ class DeviceCase:
                                                   self.w.n_q_heads, rows, self.max_len)
         return torch.zeros(n, dtype=torch.uint8, device="cuda")
 
-    def attend(self, q=None, lens=None, max_len=None, ws=None, out=None, kind=None):
+    def attend(self, q=None, lens=None, max_len=None, ws=None, out=None, kind=None, tree=None):
         q = self.q if q is None else q
         lens = self.lens if lens is None else lens
         max_len = self.max_len if max_len is None else max_len
         W = q.shape[1]
         ws = self.workspace(W) if ws is None else ws
         out = torch.empty(q.shape, dtype=torch.float32, device="cuda") if out is None else out
+        if tree is not None:
+            t = torch.from_numpy(np.ascontiguousarray(tree, dtype=np.uint8)).cuda()
+            self.tf.tf_paged_attn_verify_tree(self.k_pool, self.v_pool, self.table, lens, q, t,
+                                              self.w.scale, out, ws, max_len)
+            return out
         if kind is None:
             kind = "decode" if W == 1 else "verify" if W <= 8 else "prompt"
         fn = {"decode": self.tf.tf_paged_attn_decode, "verify": self.tf.tf_paged_attn_verify,

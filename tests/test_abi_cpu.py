@@ -90,3 +90,13 @@ def test_verify_rows_limit_and_null_pointers(lib):
                                   None) == lib.TF_EINVAL
     assert lib.raw.tf_workspace_status(None, None, None) == lib.TF_EINVAL
     assert lib.tf_status_str(lib.TF_ENOSPACE).startswith("TF_ENOSPACE")
+
+
+def test_tree_verify_host_checks(lib):
+    pool, st = _pool(lib), _streams(lib)
+    # no mask array
+    assert lib.raw.tf_paged_attn_verify_tree(ctypes.byref(pool), ctypes.byref(st), 16, 8, 4, None,
+                                             0.1, 16, 16, 1 << 30, None) == lib.TF_EINVAL
+    # more rows than a mask byte holds
+    assert lib.raw.tf_paged_attn_verify_tree(ctypes.byref(pool), ctypes.byref(st), 16, 8, 9, 16,
+                                             0.1, 16, 16, 1 << 30, None) == lib.TF_EINVAL

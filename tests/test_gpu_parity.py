@@ -251,3 +251,97 @@ def test_hd256_needs_pages_of_128():
     with pytest.raises(tf.TFError) as e:
         dc.attend(ws=ws)
     assert e.value.status == tf.TF_EUNSUPPORTED
+
+
+# --- tree-mask verify: each window row sees the positions before the window
+# and the window rows its mask names (its ancestors in a draft tree)
+
+def run_tree_parity(w, lens, rows, tree, table=None, n_pages=None):
+    case = synth.make_case(w, lens=lens, rows=rows, table=table, n_pages=n_pages)
+    dc = DeviceCase(case)
+    out = dc.attend(tree=tree)
+    torch.cuda.synchronize()
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, rows, w.group, w.scale,
+                        threads=8, tree=tree)
+    assert torch.isfinite(out).all()
+    err = max_abs(out, ref)
+    assert err <= TOL, err
+    return case, dc, out
+
+
+@pytest.mark.parametrize("d,G", [(128, 4), (128, 8), (128, 12), (128, 16), (256, 8), (512, 8),
+                                 (512, 16)])
+@pytest.mark.parametrize("W", [2, 5, 8])
+def test_tree_parity_sweep(d, G, W):
+    w = small_workload(d, G, 512, W, seed=10000 + d + 10 * G + W)
+    lens = [1024, 1537, 1023, W, W + 130]
+    tree = synth.tree_masks((10001, d, G, W), len(lens), W)
+    run_tree_parity(w, lens, W, tree)
+
+
+def test_tree_chain_masks_match_the_causal_window():
+    w = small_workload(128, 8, 512, 8, seed=10100)
+    lens = [3000, 900]
+    case, dc, out = run_tree_parity(w, lens, 8, synth.chain_masks(2, 8))
+    causal = dc.attend()
+    assert (out - causal).abs().max().item() <= TOL
+
+
+def test_tree_masks_naming_later_rows():
+    """Masks are read as given: a row may also name rows after it."""
+    rng = np.random.default_rng(10200)
+    W = 6
+    lens = [W, 700, 2049]
+    tree = rng.integers(0, 256, size=(3, W)).astype(np.uint8)
+    for r in range(W):
+        tree[:, r] |= np.uint8(1 << r)
+    w = small_workload(128, 4, 512, W, seed=10201)
+    run_tree_parity(w, lens, W, tree)
+
+
+def test_tree_paged_equals_identity_table_bytes_and_repeats():
+    w = small_workload(512, 8, 512, 4, seed=10300, sigma=0.5)
+    lens = [2000, 513, 4096]
+    tree = synth.tree_masks((10301,), 3, 4)
+    case = synth.make_case(w, lens=lens)
+    dc = DeviceCase(case)
+    a = dc.attend(tree=tree)
+    b = dc.attend(tree=tree)
+    assert torch.equal(a, b)
+    table, n_pages = synth.identity_table(case.lens, w.page_size)
+    c = DeviceCase(case, table=table, n_pages=n_pages).attend(tree=tree)
+    assert torch.equal(a, c)
+
+
+@pytest.mark.parametrize("d,G,W", [(128, 8, 8), (512, 8, 4)])
+def test_tree_split_one_long_stream(d, G, W):
+    w = synth.Workload("one", 0, 1, G, d, 512, W, seed=10400 + d + W)
+    tree = synth.tree_masks((10401, d), 1, W)
+    run_tree_parity(w, [40000 if d == 128 else 12000], W, tree)
+
+
+def test_tree_growing_scores():
+    W = 8
+    w = small_workload(128, 8, 512, W, seed=10500)
+    case = synth.make_case(w, lens=[3000, 1300 + W], rows=W)
+    for s, n in enumerate(case.lens):
+        ramp = (1.0 + 14.0 * np.arange(n) / n).astype(np.float32)[:, None, None]
+        case.k_lin[s] = synth.bf16_from_f32(synth.f32_from_bf16(case.k_lin[s]) * ramp)
+    tree = synth.tree_masks((10501,), 2, W)
+    dc = DeviceCase(case)
+    out = dc.attend(tree=tree)
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, W, w.group, w.scale,
+                        threads=8, tree=tree)
+    assert torch.isfinite(out).all()
+    assert max_abs(out, ref) <= TOL
+
+
+def test_tree_needs_pages_of_128():
+    import verify_paged_gqa_b200 as tf
+    w = small_workload(128, 4, 64, 4, seed=10600)
+    case = synth.make_case(w, lens=[300], rows=4)
+    dc = DeviceCase(case)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tf.TFError) as e:
+        dc.attend(ws=ws, tree=synth.tree_masks((10601,), 1, 4))
+    assert e.value.status == tf.TF_EUNSUPPORTED

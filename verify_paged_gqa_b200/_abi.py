@@ -79,6 +79,9 @@ for _name in ("tf_paged_attn_verify", "tf_paged_attn_prompt"):
     getattr(raw, _name).argtypes = [_P(tf_kv_pool), _P(tf_streams), _vp, _i32, _i32, _f32,
                                     _vp, _vp, _sz, _vp]
     getattr(raw, _name).restype = ctypes.c_int
+raw.tf_paged_attn_verify_tree.argtypes = [_P(tf_kv_pool), _P(tf_streams), _vp, _i32, _i32, _vp,
+                                          _f32, _vp, _vp, _sz, _vp]
+raw.tf_paged_attn_verify_tree.restype = ctypes.c_int
 raw.tf_workspace_status.argtypes = [_vp, _P(ctypes.c_uint32), _vp]
 raw.tf_workspace_status.restype = ctypes.c_int
 raw.tf_status_str.argtypes = [ctypes.c_int]
@@ -151,7 +154,7 @@ def tf_paged_attn_workspace_bytes(k_pool, v_pool, table, lens, n_q_heads, rows, 
 
 
 def _attn(fn, name, k_pool, v_pool, table, lens, q, scale, out, workspace, max_len, stream,
-          with_rows):
+          with_rows, tree=None):
     _need(q, torch.bfloat16, 4, "q")
     _need(out, torch.float32, 4, "out")
     if tuple(out.shape) != tuple(q.shape):
@@ -163,6 +166,8 @@ def _attn(fn, name, k_pool, v_pool, table, lens, q, scale, out, workspace, max_l
     args = [ctypes.byref(pool), ctypes.byref(st), q.data_ptr(), q.shape[2]]
     if with_rows:
         args.append(q.shape[1])
+    if tree is not None:
+        args.append(tree.data_ptr())
     args += [float(scale), out.data_ptr(), workspace.data_ptr(), ws_bytes, _stream(stream)]
     _check(fn(*args), name)
     return out
@@ -182,6 +187,19 @@ def tf_paged_attn_verify(k_pool, v_pool, table, lens, q, scale, out, workspace, 
     """A causal window of q.shape[1] <= 8 rows per stream."""
     return _attn(raw.tf_paged_attn_verify, "tf_paged_attn_verify", k_pool, v_pool, table, lens,
                  q, scale, out, workspace, max_len, stream, with_rows=True)
+
+
+def tf_paged_attn_verify_tree(k_pool, v_pool, table, lens, q, tree, scale, out, workspace,
+                              max_len, stream=None):
+    """A window of q.shape[1] <= 8 rows per stream under draft-tree masks:
+    tree is a uint8 [S][rows] device tensor, bit c of tree[s][r] set when row r
+    sees window row c (positions before the window are seen by every row)."""
+    _need(tree, torch.uint8, 2, "tree")
+    if tuple(tree.shape) != (q.shape[0], q.shape[1]):
+        raise ValueError("tree must be [S][rows]")
+    return _attn(raw.tf_paged_attn_verify_tree, "tf_paged_attn_verify_tree", k_pool, v_pool,
+                 table, lens, q, scale, out, workspace, max_len, stream, with_rows=True,
+                 tree=tree)
 
 
 def tf_paged_attn_prompt(k_pool, v_pool, table, lens, q, scale, out, workspace, max_len,

@@ -88,6 +88,7 @@ struct PmSmem {
     alignas(16) float lsum[NR];   // row sums (inverted for a finished row block)
     alignas(16) float red[4][NR];
     long long rowoff[2][NR];      // output offset of row r (by segment parity); -1 past M
+    uint32_t rowvis[NR / 32][8];  // tree masks: bit r of [h][c] -- row 32 h + r sees window row c
     CtaRange range;               // this CTA's tiles
     uint64_t full[C::NU];
     uint64_t empty[C::NU];
@@ -252,12 +253,22 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
     (void)mbar_wait(&sm.fin, 0);
 }
 
+// Whether the thread's row R0 + r sees its position (see the tile loop).
+template <bool kTree>
+__device__ __forceinline__ bool pm_sees(int r, int rvis, uint32_t vis)
+{
+    if constexpr (kTree)
+        return ((vis >> r) & 1u) != 0;
+    else
+        return r >= rvis;
+}
+
 // ---- softmax warps -----------------------------------------------------------
 
 // NW = 4 * NR / 32 softmax warps: warp w reads tensor-memory lanes
 // 32 * (w % 4) .. + 31 (tile positions, or O^T dims), and owns the 32 rows
 // [32 h, 32 h + 32) with h = (w - 2) / 4.
-template <int D, int NR>
+template <int D, int NR, bool kTree>
 __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, int warp, int lane)
 {
     using C = PmCfg<D, NR>;
@@ -340,6 +351,20 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                     }
                 }
             }
+            if (kTree && st < NR / 32 * 8) {
+                // the block's rows that see window row c, from the stream's masks
+                const int hh = st >> 3, c = st & 7;
+                uint32_t wv = 0;
+                if (c < p.W) {
+                    const uint8_t *tm = p.tree + (size_t)it.s * p.W;
+                    for (int r = 0; r < 32; ++r) {
+                        const int m = it.b * NR + 32 * hh + r;
+                        if (m < p.M && ((__ldg(tm + m / p.G) >> c) & 1))
+                            wv |= 1u << r;
+                    }
+                }
+                sm.rowvis[hh][c] = wv;
+            }
             fence_async_smem();
             named_barrier(1, NT);
             if (st == 0)
@@ -350,19 +375,30 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
 #pragma unroll
         for (int r = 0; r < 32; ++r)
             l[r] = 0.f;
-        // the block's first row sees the fewest positions
-        const int lim_lo = row_lim(p, it.len, it.b * NR);
+        // the block's first row sees the fewest positions (under tree masks,
+        // every row sees the positions before the window)
+        const int lim_lo = kTree ? it.len - p.W : row_lim(p, it.len, it.b * NR);
         for (int t = 0; t < n; ++t) {
             const uint32_t u = u0 + t;
             const int tpos = it.key0 + t * PT;
             const uint32_t tS = lane_base + C::kColS + (u & 1u) * NR + R0;
             // a tile every row of the block sees whole needs no mask
             const bool whole = tpos + PT <= lim_lo && tpos + PT <= it.key1;
-            // rows R0 + r, r >= rvis, see this thread's position
+            // causal: rows R0 + r, r >= rvis, see this thread's position;
+            // tree: row R0 + r sees it when bit r of vis is set
             const int pos = tpos + tid;
-            const int rvis = (pos >= it.key1 || pos >= it.len)
-                                 ? 32
-                                 : p.G * max(0, pos - (it.len - p.W)) - it.b * NR - R0;
+            int rvis = 32;
+            uint32_t vis = 0;
+            if constexpr (kTree) {
+                const int c = pos - (it.len - p.W);
+                vis = (pos >= it.key1 || pos >= it.len) ? 0u
+                      : c < 0                         ? 0xffffffffu
+                                                      : sm.rowvis[h][c];
+            } else {
+                rvis = (pos >= it.key1 || pos >= it.len)
+                           ? 32
+                           : p.G * max(0, pos - (it.len - p.W)) - it.b * NR - R0;
+            }
             ok = pwait(sm, &sm.s_full[u & 1u], (u >> 1) & 1u, p.flags, kWaitFull) && ok;
             tc_fence_after();
 
@@ -382,7 +418,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                 if (!whole) {
 #pragma unroll
                     for (int r = 0; r < 32; ++r)
-                        x[r] = r >= rvis ? x[r] : NEG_INF;
+                        x[r] = pm_sees<kTree>(r, rvis, vis) ? x[r] : NEG_INF;
                 }
 #pragma unroll
                 for (int r = 0; r < 32; ++r)
@@ -395,7 +431,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                 load_scores<32>(tS, y);
 #pragma unroll
                 for (int r = 0; r < 32; ++r)
-                    y[r] = (whole || r >= rvis) ? y[r] * sl : NEG_INF;
+                    y[r] = (whole || pm_sees<kTree>(r, rvis, vis)) ? y[r] * sl : NEG_INF;
                 xpose_reduce<32, true>(y, lane);
                 sm.red[wq][R0 + lane] = y[0];
                 named_barrier(1, NT);
@@ -450,7 +486,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
                 if (!whole) {
 #pragma unroll
                     for (int r = 0; r < 32; ++r)
-                        x[r] = r >= rvis ? x[r] : NEG_INF;
+                        x[r] = pm_sees<kTree>(r, rvis, vis) ? x[r] : NEG_INF;
                 }
             }
             // --- V rows past the stream's end: zero them (0 * NaN = NaN) ----
@@ -566,7 +602,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
     }
 }
 
-template <int D, int NR>
+template <int D, int NR, bool kTree>
 __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     attn_pm_kernel(const __grid_constant__ PmArgs a)
 {
@@ -614,7 +650,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
             pm_issuer<D, NR>(a, sm);
         __syncwarp();
     } else {
-        pm_softmax<D, NR>(a, sm, warp, lane);
+        pm_softmax<D, NR, kTree>(a, sm, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -626,7 +662,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     }
 }
 
-template <int D, int NR>
+template <int D, int NR, bool kTree>
 cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
 {
     PmArgs a;
@@ -642,43 +678,51 @@ cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
         return cudaErrorInvalidDevice;
     constexpr size_t bytes = pm_smem_bytes<D, NR>();
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(attn_pm_kernel<D, NR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(attn_pm_kernel<D, NR, kTree>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)bytes);
         if (e != cudaSuccess)
             return e;
         configured[dev] = true;
     }
-    attn_pm_kernel<D, NR><<<grid, PmCfg<D, NR>::kThreads, bytes, stream>>>(a);
+    attn_pm_kernel<D, NR, kTree><<<grid, PmCfg<D, NR>::kThreads, bytes, stream>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 // Rows per row block, or 0 when this kernel does not take the call: tiles
-// stay inside a page, and blocks of more than 64 rows at head dim 128 go to
-// the row-major tensor-core kernel.
+// stay inside a page, and causal blocks of more than 64 rows at head dim 128
+// go to the row-major tensor-core kernel (tree calls run here with several
+// row blocks).
 int pm_rows(const AttnParams &p)
 {
     if (p.P % PT != 0 || !pool_rows_fit(p))
         return 0;
     if (p.D == 128)
-        return p.M <= 32 ? 32 : p.M <= 64 ? 64 : 0;
+        return p.M <= 32 ? 32 : (p.M <= 64 || p.has_tree) ? 64 : 0;
     if (p.D == 256 || p.D == 512)
         return 32;
     return 0;
 }
 
-cudaError_t launch_attn_pm(const AttnParams &p, int grid, cudaStream_t stream)
+template <bool kTree>
+cudaError_t launch_attn_pm_t(const AttnParams &p, int grid, cudaStream_t stream)
 {
     if (p.D == 128 && p.RB == 32)
-        return launch_pm<128, 32>(p, grid, stream);
+        return launch_pm<128, 32, kTree>(p, grid, stream);
     if (p.D == 128 && p.RB == 64)
-        return launch_pm<128, 64>(p, grid, stream);
+        return launch_pm<128, 64, kTree>(p, grid, stream);
     if (p.D == 256 && p.RB == 32)
-        return launch_pm<256, 32>(p, grid, stream);
+        return launch_pm<256, 32, kTree>(p, grid, stream);
     if (p.D == 512 && p.RB == 32)
-        return launch_pm<512, 32>(p, grid, stream);
+        return launch_pm<512, 32, kTree>(p, grid, stream);
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attn_pm(const AttnParams &p, int grid, cudaStream_t stream)
+{
+    return p.has_tree ? launch_attn_pm_t<true>(p, grid, stream)
+                      : launch_attn_pm_t<false>(p, grid, stream);
 }
 
 }  // namespace tfp

@@ -41,6 +41,7 @@ struct AttnParams {
     const int32_t *table;
     const int32_t *lens;
     const __nv_bfloat16 *q;
+    const uint8_t *tree;  // tree-verify row masks [S][W] (bit c: the row sees window row c), or null
     float *out;
     float *part;        // split-context partials (workspace past the header)
     uint32_t *flags;    // workspace status word
@@ -52,6 +53,7 @@ struct AttnParams {
     int32_t n_cta;              // persistent CTAs of the partial kernel (the work split)
     int32_t VT;                 // entry tiles of work in front of every unit
     int32_t whole;              // 1: CTA c takes unit c whole (no split, no partials)
+    int32_t has_tree;           // 1: tree-verify call (the tree pointer holds the masks)
     long long *first_tile;      // workspace: where each stream's work starts in the launch
     long long *total_tiles;     // workspace: work tiles of the launch
     float scale_log2;           // scale * log2(e): scores are kept in log2 units

@@ -39,14 +39,18 @@ __host__ __device__ __forceinline__ bool len_ok(const AttnParams &p, int len)
     return len >= p.W && len <= p.max_len && (int64_t)len <= (int64_t)p.table_stride * p.P;
 }
 
-// One past the last position any row of row block b may see.
+// One past the last position any row of row block b may see (under tree
+// masks a row may see any row of its window).
 __host__ __device__ __forceinline__ int block_lim(const AttnParams &p, int len, int b)
 {
+    if (p.has_tree)
+        return len;
     const int m_last = min(p.M, (b + 1) * p.RB) - 1;
     return len - p.W + m_last / p.G + 1;
 }
 
-// One past the position row m sees (rows past M are clamped to the last row).
+// One past the position row m sees (rows past M are clamped to the last row);
+// causal windows only.
 __host__ __device__ __forceinline__ int row_lim(const AttnParams &p, int len, int m)
 {
     return len - p.W + min(m, p.M - 1) / p.G + 1;

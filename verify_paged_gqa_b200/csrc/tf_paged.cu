@@ -85,7 +85,7 @@ struct Plan {
 };
 
 int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t rows,
-              int32_t rows_max, Plan *plan)
+              int32_t rows_max, bool tree, Plan *plan)
 {
     int rc = check_pool_streams(pool, st);
     if (rc != TF_OK)
@@ -116,13 +116,21 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     p.G = G;
     p.W = rows;
     p.M = static_cast<int32_t>(M);
+    p.has_tree = tree ? 1 : 0;
     // More than one CUDA-core row block of rows sharing a KV head: a dense
     // QK^T / PV tile for the tensor cores.  Up to 64 rows (128 at head dim
     // 512 in blocks of 32) go with the positions on the MMA's M; larger
     // blocks with the rows there.
     plan->kernel = Kernel::kSimt;
     p.RB = kSimtRows;
-    if (p.D == 256) {
+    if (tree) {
+        // tree masks run on the position-major kernel only (any row count)
+        const int nr = pm_rows(p);
+        if (nr == 0)
+            return TF_EUNSUPPORTED;
+        plan->kernel = Kernel::kPm;
+        p.RB = nr;
+    } else if (p.D == 256) {
         // head dim 256 runs on the position-major kernel only (any row count)
         const int nr = pm_rows(p);
         if (nr == 0)
@@ -167,11 +175,11 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
 }
 
 int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32_t Hq,
-              int32_t rows, int32_t rows_max, float scale, float *out, void *ws,
-              size_t ws_bytes, void *stream)
+              int32_t rows, int32_t rows_max, const uint8_t *tree, float scale, float *out,
+              void *ws, size_t ws_bytes, void *stream)
 {
     Plan plan;
-    int rc = make_plan(pool, st, Hq, rows, rows_max, &plan);
+    int rc = make_plan(pool, st, Hq, rows, rows_max, tree != nullptr, &plan);
     if (rc != TF_OK)
         return rc;
     if (!q || !out || !ws || !aligned16(q) || !aligned16(out) || !aligned16(ws))
@@ -188,6 +196,7 @@ int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32
     p.table = st->table;
     p.lens = st->lens;
     p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.tree = tree;
     p.out = out;
     char *wsb = static_cast<char *>(ws);
     p.flags = reinterpret_cast<uint32_t *>(wsb);
@@ -259,24 +268,41 @@ size_t tf_paged_attn_workspace_bytes(const tf_kv_pool *pool, const tf_streams *s
                                      int32_t n_q_heads, int32_t rows)
 {
     Plan plan;
-    if (make_plan(pool, streams, n_q_heads, rows, 4096, &plan) != TF_OK)
+    if (make_plan(pool, streams, n_q_heads, rows, 4096, false, &plan) != TF_OK)
         return 0;
-    return plan.ws_bytes;
+    size_t bytes = plan.ws_bytes;
+    // enough for a tree-verify call with the same arguments too
+    Plan tp;
+    if (rows <= 8 && make_plan(pool, streams, n_q_heads, rows, 8, true, &tp) == TF_OK &&
+        tp.ws_bytes > bytes)
+        bytes = tp.ws_bytes;
+    return bytes;
 }
 
 int tf_paged_attn_decode(const tf_kv_pool *pool, const tf_streams *streams, const void *q,
                          int32_t n_q_heads, float scale, float *out, void *workspace,
                          size_t workspace_bytes, void *stream)
 {
-    return attn_call(pool, streams, q, n_q_heads, 1, 1, scale, out, workspace, workspace_bytes,
-                     stream);
+    return attn_call(pool, streams, q, n_q_heads, 1, 1, nullptr, scale, out, workspace,
+                     workspace_bytes, stream);
 }
 
 int tf_paged_attn_verify(const tf_kv_pool *pool, const tf_streams *streams, const void *q,
                          int32_t n_q_heads, int32_t rows, float scale, float *out,
                          void *workspace, size_t workspace_bytes, void *stream)
 {
-    return attn_call(pool, streams, q, n_q_heads, rows, 8, scale, out, workspace,
+    return attn_call(pool, streams, q, n_q_heads, rows, 8, nullptr, scale, out, workspace,
+                     workspace_bytes, stream);
+}
+
+int tf_paged_attn_verify_tree(const tf_kv_pool *pool, const tf_streams *streams, const void *q,
+                              int32_t n_q_heads, int32_t rows, const uint8_t *tree_masks,
+                              float scale, float *out, void *workspace, size_t workspace_bytes,
+                              void *stream)
+{
+    if (!tree_masks)
+        return TF_EINVAL;
+    return attn_call(pool, streams, q, n_q_heads, rows, 8, tree_masks, scale, out, workspace,
                      workspace_bytes, stream);
 }
 
@@ -284,7 +310,7 @@ int tf_paged_attn_prompt(const tf_kv_pool *pool, const tf_streams *streams, cons
                          int32_t n_q_heads, int32_t rows, float scale, float *out,
                          void *workspace, size_t workspace_bytes, void *stream)
 {
-    return attn_call(pool, streams, q, n_q_heads, rows, 4096, scale, out, workspace,
+    return attn_call(pool, streams, q, n_q_heads, rows, 4096, nullptr, scale, out, workspace,
                      workspace_bytes, stream);
 }
 
@@ -371,7 +397,7 @@ extern "C" int tf_paged_attn_decode_noalloc(const tf_kv_pool *pool, const tf_str
 {
     using namespace tfp;
     Plan plan;
-    int rc = make_plan(pool, streams, n_q_heads, 1, 1, &plan);
+    int rc = make_plan(pool, streams, n_q_heads, 1, 1, false, &plan);
     if (rc != TF_OK)
         return rc;
     if (!q || !out || !aligned16(q) || !aligned16(out) || !std::isfinite(scale))
@@ -390,6 +416,6 @@ extern "C" int tf_paged_attn_decode_noalloc(const tf_kv_pool *pool, const tf_str
     // they are read.
     if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess)
         return TF_ECUDA;
-    return attn_call(pool, streams, q, n_q_heads, 1, 1, scale, out, ws, kStaticScratchBytes,
+    return attn_call(pool, streams, q, n_q_heads, 1, 1, nullptr, scale, out, ws, kStaticScratchBytes,
                      stream);
 }
