@@ -598,7 +598,8 @@ def main():
         # the shape variants the pages mention (GQA 12, GQA 16 at head dim 512,
         # head dim 256), each timed the same way
         line["variants"] = []
-        for name in ("gqa12_verify", "gqa16_hd512_decode", "hd256_verify", "tree_verify_4x131k"):
+        for name in ("gqa12_verify", "gqa16_hd512_decode", "hd256_verify", "tree_verify_4x131k",
+                     "decode_12x40k_p37"):
             line["variants"].append(measure_other(name, args, barrier, dist, world, local))
             torch.cuda.empty_cache()
 

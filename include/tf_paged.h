@@ -89,8 +89,12 @@ extern "C" {
 #define TF_DEV_TIMEOUT 4u   /* a pipeline wait gave up (an internal error) */
 
 /* The pool: K and V pages, device memory, 16-byte aligned.
- * page_size must be a multiple of 64; head_dim must be 128, 256 or 512
- * (head dim 256 also needs page_size a multiple of 128). */
+ * page_size may be any positive size (TensorFold #1620, Checks, the kernel-
+ * contract bullet: the paged prompt kernel is checked over pages of 512, 37
+ * and 64); head_dim must be 128, 256 or 512.  The tensor-core kernels need
+ * page_size a multiple of 128: other sizes run on the CUDA-core kernel,
+ * whose tiles may then straddle pages, and head dim 256 and tree-mask calls
+ * are refused for them (TF_EUNSUPPORTED). */
 typedef struct tf_kv_pool {
     void *k_pool;
     void *v_pool;

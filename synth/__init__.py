@@ -28,6 +28,8 @@ Workloads (synthetic stand-ins for the pages' served runs):
     head dim 512 global layer, four-row cells);
   * ``prompt_9216``    one 9,216-token prompt written into shuffled pages, then
     attended in causal chunks of 512 rows, 8 KV / 32 query heads, d 128;
+  * ``decode_12x40k_p37`` the decode workload in pages of 37 positions
+    (TensorFold #1620, Checks: the paged prompt kernel over pages of 37);
   * ``tree_verify_4x131k`` the verify workload with every stream's window a
     random draft tree (TensorFold #1620 calls the verify kernels "tree
     attention"; each row sees its ancestors and itself).
@@ -146,6 +148,9 @@ WORKLOADS = {
     # the verify workload with each stream's 8 rows a random draft tree
     "tree_verify_4x131k": Workload("tree_verify_4x131k", 4, 4, 8, 128, 512, 8, seed=11,
                                    lens=(131072,) * 4, tree=True),
+    # the decode workload in pages of 37 positions (tiles straddle pages)
+    "decode_12x40k_p37": Workload("decode_12x40k_p37", 12, 8, 4, 128, 37, 1, seed=12,
+                                  lens=(40960,) * 12),
     # smaller copies of the decode and verify workloads for profiler captures
     # (still larger than the 126 MB L2)
     "decode_12x8k": Workload("decode_12x8k", 12, 8, 4, 128, 512, 1, seed=6, lens=(8192,) * 12),
@@ -178,7 +183,7 @@ def workload_tree(w: Workload, n_streams: int | None = None, rows: int | None = 
     """The tree masks of a tree workload (None for a causal one)."""
     if not w.tree:
         return None
-    return tree_masks((w.seed, 7), w.n_streams if n_streams is None else n_streams,
+    return tree_masks((w.seed, 11), w.n_streams if n_streams is None else n_streams,
                       w.rows if rows is None else rows)
 
 

@@ -62,7 +62,7 @@ def _streams(lib, **kw):
 
 @pytest.mark.parametrize("pool_kw,streams_kw,hq,rows,want", [
     ({"head_dim": 64}, {}, 8, 1, "TF_EUNSUPPORTED"),
-    ({"page_size": 100}, {}, 8, 1, "TF_EUNSUPPORTED"),
+    ({"page_size": 0}, {}, 8, 1, "TF_EINVAL"),
     ({"n_pages": 0}, {}, 8, 1, "TF_EINVAL"),
     ({}, {"max_len": 2049}, 8, 1, "TF_EINVAL"),          # past table_stride * page_size
     ({}, {}, 7, 1, "TF_EINVAL"),                          # query heads not a multiple

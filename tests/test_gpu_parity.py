@@ -345,3 +345,71 @@ def test_tree_needs_pages_of_128():
     with pytest.raises(tf.TFError) as e:
         dc.attend(ws=ws, tree=synth.tree_masks((10601,), 1, 4))
     assert e.value.status == tf.TF_EUNSUPPORTED
+
+
+# --- any page size (the pages check the paged prompt kernel over pages of 37):
+# tiles of the CUDA-core kernel straddle pages, one bulk copy per page piece
+
+@pytest.mark.parametrize("P", [37, 1, 3, 100, 509])
+@pytest.mark.parametrize("d", [128, 512])
+@pytest.mark.parametrize("W", [1, 4, 8])
+def test_parity_any_page_size(P, d, W):
+    w = small_workload(d, 4, P, W, seed=11000 + P + d + W)
+    lens = [P * 7, P * 3 + 1, W + 2, 1000] if P > 1 else [40, 9, W, 300]
+    run_parity(w, lens, W)
+
+
+@pytest.mark.parametrize("W", [16, 100])
+def test_parity_prompt_page37(W):
+    w = small_workload(128, 4, 37, W, seed=11100 + W)
+    run_parity(w, [W, W + 300, 700], W)
+
+
+def test_page37_paged_equals_identity_table_and_put_rows_bit_exact():
+    w = small_workload(128, 8, 37, 2, seed=11200)
+    lens = [2000, 37, 38, 75]
+    case = synth.make_case(w, lens=lens)
+    a = DeviceCase(case).attend()
+    table, n_pages = synth.identity_table(case.lens, w.page_size)
+    b = DeviceCase(case, table=table, n_pages=n_pages).attend()
+    assert torch.equal(a, b)
+    # the row write over pages of 37 and of 1
+    import verify_paged_gqa_b200 as tf
+    rng = np.random.default_rng(11201)
+    for P in (37, 1):
+        wp = synth.Workload("put", 3, 2, 4, 128, P, 3, seed=11202 + P)
+        lens = np.array([3, P + 3, 5 * P + 2], dtype=np.int32)
+        table, n_pages, _ = synth.page_table(wp, lens)
+        host_k = rng.integers(0, 0x7F7F, size=(n_pages, 2, P, 128)).astype(np.uint16)
+        host_v = host_k[::-1].copy()
+        kp, vp = bf16_tensor(host_k), bf16_tensor(host_v)
+        kr = rng.integers(0, 0xFFFF, size=(3, 3, 2, 128)).astype(np.uint16)
+        vr = rng.integers(0, 0xFFFF, size=(3, 3, 2, 128)).astype(np.uint16)
+        tf.tf_kv_put_rows(kp, vp, torch.from_numpy(table).cuda(), torch.from_numpy(lens).cuda(),
+                          bf16_tensor(kr), bf16_tensor(vr), max_len=int(lens.max()))
+        oracle.put_rows(host_k, host_v, table, lens, kr, vr)
+        assert np.array_equal(kp.view(torch.int16).cpu().numpy().view(np.uint16), host_k)
+        assert np.array_equal(vp.view(torch.int16).cpu().numpy().view(np.uint16), host_v)
+
+
+def test_page37_bad_page_is_flagged_and_shapes_refused():
+    import verify_paged_gqa_b200 as tf
+    w = small_workload(128, 4, 37, 1, seed=11300)
+    case = synth.make_case(w, lens=[500, 90])
+    dc = DeviceCase(case)
+    ws = dc.workspace(1)
+    tf.tf_workspace_status(ws)
+    dc.table[0, 3] = dc.k_pool.shape[0] + 2      # a page in the middle of a straddling tile
+    dc.attend(ws=ws)
+    assert tf.tf_workspace_status(ws) & tf.TF_DEV_BAD_PAGE
+    # head dim 256 and tree masks need pages that are a multiple of 128
+    w2 = small_workload(256, 4, 37, 4, seed=11301)
+    dc2 = DeviceCase(synth.make_case(w2, lens=[300], rows=4))
+    ws2 = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tf.TFError) as e:
+        dc2.attend(ws=ws2)
+    assert e.value.status == tf.TF_EUNSUPPORTED
+    dc3 = DeviceCase(synth.make_case(w, lens=[300], rows=4))
+    with pytest.raises(tf.TFError) as e:
+        dc3.attend(ws=ws2, q=dc3.q, tree=synth.tree_masks((11302,), 1, 4))
+    assert e.value.status == tf.TF_EUNSUPPORTED

@@ -387,18 +387,12 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
             // causal: rows R0 + r, r >= rvis, see this thread's position;
             // tree: row R0 + r sees it when bit r of vis is set
             const int pos = tpos + tid;
-            int rvis = 32;
-            uint32_t vis = 0;
-            if constexpr (kTree) {
-                const int c = pos - (it.len - p.W);
-                vis = (pos >= it.key1 || pos >= it.len) ? 0u
-                      : c < 0                         ? 0xffffffffu
-                                                      : sm.rowvis[h][c];
-            } else {
-                rvis = (pos >= it.key1 || pos >= it.len)
-                           ? 32
-                           : p.G * max(0, pos - (it.len - p.W)) - it.b * NR - R0;
-            }
+            const int rvis = kTree || pos >= it.key1 || pos >= it.len
+                                 ? 32
+                                 : p.G * max(0, pos - (it.len - p.W)) - it.b * NR - R0;
+            const uint32_t vis = !kTree || pos >= it.key1 || pos >= it.len ? 0u
+                                 : pos < it.len - p.W                     ? 0xffffffffu
+                                                       : sm.rowvis[h][pos - (it.len - p.W)];
             ok = pwait(sm, &sm.s_full[u & 1u], (u >> 1) & 1u, p.flags, kWaitFull) && ok;
             tc_fence_after();
 

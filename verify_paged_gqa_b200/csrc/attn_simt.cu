@@ -218,6 +218,53 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
         if (have_nx && producer_q<D>(p, sm, nx, j + 1, pol))
             q_issued = j + 2;
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
+        if (p.P % TK != 0) {
+            // Any page size: a tile of TK positions may straddle pages, and is
+            // filled by one bulk copy per page piece (its rows land in order).
+            // The page walk moves forward piece by piece; the next page id is
+            // read one page ahead.  A piece on a page outside the pool is not
+            // read: its bytes are released with complete_tx (and flagged).
+            int lp = it.key0 / p.P;
+            int page_end = (lp + 1) * p.P;
+            int32_t page = __ldg(trow + lp);
+            int32_t page_nx = page_end < it.key1 ? __ldg(trow + lp + 1) : 0;
+            for (int t0 = it.key0; t0 < it.key1 && !sm.abort_flag; t0 += TK, ++T) {
+                const int stage = T % NSTAGE;
+                if (!wait_or_abort(sm, &sm.empty[stage], ((T / NSTAGE) & 1u) ^ 1u, p.flags, kWaitEmpty))
+                    break;
+                sm.stage_tile[stage] = T;
+                const int t1 = min(t0 + TK, it.key1);
+                mbar_arrive_expect_tx(&sm.full[stage], 2u * static_cast<uint32_t>(t1 - t0) * D * 2u);
+                for (int pos = t0; pos < t1;) {
+                    const int n = min(page_end, t1) - pos;
+                    const uint32_t nb = static_cast<uint32_t>(n) * D * 2u;
+                    if (page >= 0 && page < p.n_pages) {
+                        const size_t off =
+                            (((size_t)page * p.Hkv + it.kh) * p.P + (pos - (page_end - p.P))) * D;
+                        bulk_g2s(sm.kv[stage][0] + (pos - t0) * D * 2, p.k_pool + off, nb,
+                                 &sm.full[stage], pol);
+                        bulk_g2s(sm.kv[stage][1] + (pos - t0) * D * 2, p.v_pool + off, nb,
+                                 &sm.full[stage], pol);
+                    } else {
+                        set_flag(p.flags, kDevBadPage);
+                        mbar_complete_tx(&sm.full[stage], 2u * nb);
+                    }
+                    pos += n;
+                    if (pos == page_end) {
+                        ++lp;
+                        page_end += p.P;
+                        page = page_nx;
+                        if (page_end < it.key1)   // page lp + 1 holds keys of this segment
+                            page_nx = __ldg(trow + lp + 1);
+                    }
+                }
+            }
+            have = have_nx;
+            it = nx;
+            cur = ahead;
+            ++j;
+            continue;
+        }
         const int lp_end = (it.key1 + p.P - 1) / p.P;
         for (int lp = it.key0 / p.P; lp < lp_end && !sm.abort_flag; ++lp) {
             const int32_t page = page_next;

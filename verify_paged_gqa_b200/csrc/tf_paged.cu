@@ -41,8 +41,6 @@ int check_pool_streams(const tf_kv_pool *pool, const tf_streams *st)
         return TF_EINVAL;
     if (pool->head_dim != 128 && pool->head_dim != 256 && pool->head_dim != 512)
         return TF_EUNSUPPORTED;
-    if (pool->page_size % 64 != 0)
-        return TF_EUNSUPPORTED;
     if (st->n_streams < 0 || st->table_stride < 1 || st->max_len < 1)
         return TF_EINVAL;
     if ((int64_t)st->max_len > (int64_t)st->table_stride * pool->page_size)
