@@ -17,6 +17,8 @@ Sources for what is computed:
   * TensorFold pull request #2730 (eight-row verify window), "What this
     changes" and the checklist: a window is the pending token plus drafts,
     and drafted output equals undrafted output (causal inside the window).
+  * TensorFold pull request #1620, opening comment, "Kept states" bullet: a
+    kept state is copied by walking the slot's pages (``copy_state``).
   * TensorFold pull request #1620, opening comment, first bullet and Reads
     bullet: the verify kernels are "tree attention" over key groups of one
     page.  The pages give no mask; the reading is a per-row bitmask over the
@@ -69,6 +71,9 @@ def open_library(path: str):
     lib.tfo_attend_units_tree.restype = ctypes.c_int
     lib.tfo_put_rows.argtypes = [p, p, i32, i32, i32, i32, p, i32, p, i32, p, p, i32]
     lib.tfo_put_rows.restype = ctypes.c_int
+    lib.tfo_copy_state.argtypes = [p, p, i32, i32, p, i32, p, p, i32, i32, p, i32, i32, i32, p,
+                                   i32]
+    lib.tfo_copy_state.restype = ctypes.c_int
     return lib
 
 
@@ -163,3 +168,26 @@ def put_rows(k_pool, v_pool, table, lens, k_rows, v_rows, lib=None):
                           table.shape[1], _ptr(lens), S, _ptr(k_rows), _ptr(v_rows), W)
     if st != 0:
         raise ValueError(f"oracle put_rows refused its arguments (status {st})")
+
+
+def copy_state(src_k, src_v, src_table, dst_k, dst_v, dst_table, lens, lib=None):
+    """Host copy of every stream's positions [0, lens[s]) from the source pools'
+    pages to the destination pools' pages (in place in dst, bitwise).
+
+    pools : uint16 [n_pages][Hkv][P][d] (source and destination may differ in
+            n_pages and P);  tables: int32 [S][stride] each.
+    """
+    lib = lib or _load()
+    for a in (src_k, src_v, dst_k, dst_v):
+        assert a.flags.c_contiguous and a.dtype == np.uint16
+    sn, Hkv, sP, d = src_k.shape
+    dn, Hkv2, dP, d2 = dst_k.shape
+    assert (Hkv, d) == (Hkv2, d2)
+    src_table = np.ascontiguousarray(src_table, dtype=np.int32)
+    dst_table = np.ascontiguousarray(dst_table, dtype=np.int32)
+    lens = np.ascontiguousarray(lens, dtype=np.int32)
+    st = lib.tfo_copy_state(_ptr(src_k), _ptr(src_v), sn, sP, _ptr(src_table),
+                            src_table.shape[1], _ptr(dst_k), _ptr(dst_v), dn, dP,
+                            _ptr(dst_table), dst_table.shape[1], Hkv, d, _ptr(lens), len(lens))
+    if st != 0:
+        raise ValueError(f"oracle copy_state refused its arguments (status {st})")

@@ -50,6 +50,15 @@
  *
  * The row write (tfo_put_rows) is the plain host scatter: row r of stream s
  * goes to page table[s][pos / P], slot pos % P, with pos = len_s - W + r.
+ *
+ * The state copy (tfo_copy_state) follows the same page's "Kept states"
+ * bullet (opening comment): a kept state is copied by walking the slot's
+ * pages.  Reading: for every stream s, position j < len_s and KV head kh,
+ * the d values of K (and of V) at src page src_table[s][j / Ps], slot
+ * j % Ps are copied to dst page dst_table[s][j / Pd], slot j % Pd.  A
+ * linear buffer is a pool whose one page per stream holds the whole state,
+ * so keeping (pages to linear), resuming (linear to pages) and reusing
+ * pages (pages to pages) are the one copy.
  */
 #include <math.h>
 #include <pthread.h>
@@ -284,6 +293,41 @@ int tfo_put_rows(uint16_t *k_pool, uint16_t *v_pool, int32_t n_pages,
                 const int64_t src = (((int64_t)s * W + r) * Hkv + kh) * d;
                 memcpy(k_pool + dst, k_rows + src, sizeof(uint16_t) * (size_t)d);
                 memcpy(v_pool + dst, v_rows + src, sizeof(uint16_t) * (size_t)d);
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * The state copy: positions [0, lens[s]) of every KV head of every stream,
+ * from the source pool's pages to the destination pool's pages, each found
+ * through its own table.  Pools are [n_pages][Hkv][P][d] bf16 (the two may
+ * differ in n_pages and P).  Bytes are copied, never converted.
+ * Returns 0, or -1 when a position or page id falls outside its range.
+ */
+int tfo_copy_state(const uint16_t *src_k, const uint16_t *src_v, int32_t src_n_pages,
+                   int32_t src_P, const int32_t *src_table, int32_t src_stride,
+                   uint16_t *dst_k, uint16_t *dst_v, int32_t dst_n_pages, int32_t dst_P,
+                   const int32_t *dst_table, int32_t dst_stride, int32_t Hkv, int32_t d,
+                   const int32_t *lens, int32_t S)
+{
+    int32_t s, kh;
+    int64_t j;
+    for (s = 0; s < S; ++s) {
+        if (lens[s] < 0 || lens[s] > (int64_t)src_stride * src_P ||
+            lens[s] > (int64_t)dst_stride * dst_P)
+            return -1;
+        for (j = 0; j < lens[s]; ++j) {
+            const int32_t sp = src_table[(int64_t)s * src_stride + j / src_P];
+            const int32_t dp = dst_table[(int64_t)s * dst_stride + j / dst_P];
+            if (sp < 0 || sp >= src_n_pages || dp < 0 || dp >= dst_n_pages)
+                return -1;
+            for (kh = 0; kh < Hkv; ++kh) {
+                const int64_t from = (((int64_t)sp * Hkv + kh) * src_P + j % src_P) * d;
+                const int64_t to = (((int64_t)dp * Hkv + kh) * dst_P + j % dst_P) * d;
+                memcpy(dst_k + to, src_k + from, sizeof(uint16_t) * (size_t)d);
+                memcpy(dst_v + to, src_v + from, sizeof(uint16_t) * (size_t)d);
             }
         }
     }

@@ -20,7 +20,11 @@ What pins what:
   * tree masks: a hand-derived tree with siblings, brute force and torch's
     attention with the explicit mask, every tree row equal (to the bit) to a
     decode over the keys on its path, and chain masks equal to the causal
-    window.
+    window;
+  * the state copy: per-element brute force over tiny pools with different
+    page sizes (untouched bytes included), a round trip through a linear
+    buffer checked against numpy gathers, and agreement with the row write
+    putting the same rows into the same pages.
 """
 from __future__ import annotations
 
@@ -286,5 +290,86 @@ def pin_tree_paths(lib=None):
     assert np.abs(got - base).max() > 1e-3
 
 
+def _state_pool(rng, n_pages, Hkv, P, d, fill=None):
+    if fill is not None:
+        k = np.full((n_pages, Hkv, P, d), fill, dtype=np.uint16)
+        return k, k.copy()
+    return (rng.integers(0, 0x7F7F, size=(n_pages, Hkv, P, d)).astype(np.uint16),
+            rng.integers(0, 0x7F7F, size=(n_pages, Hkv, P, d)).astype(np.uint16))
+
+
+def _gather_linear(pool, table, n):
+    """Stream positions 0..n-1 of one table row, by numpy indexing: [n][Hkv][d]."""
+    P = pool.shape[2]
+    pages = np.asarray(table)[np.arange(n) // P]
+    return pool[pages, :, np.arange(n) % P, :]
+
+
+def pin_copy_state_brute(lib=None):
+    rng = np.random.default_rng(19)
+    Hkv, d = 2, 3
+    lens = np.array([7, 4, 0], dtype=np.int32)
+    sk, sv = _state_pool(rng, 9, Hkv, 3, d)
+    st = np.array([[4, 0, 7], [8, 2, 5], [1, 3, 6]], dtype=np.int32)
+    dk, dv = _state_pool(rng, 6, Hkv, 5, d, fill=synth.BF16_NAN)
+    dt = np.array([[3, 1], [0, 5], [2, 4]], dtype=np.int32)
+    oracle.copy_state(sk, sv, st, dk, dv, dt, lens, lib=lib)
+    want_k = np.full_like(dk, synth.BF16_NAN)
+    want_v = want_k.copy()
+    for s in range(3):
+        for j in range(int(lens[s])):
+            for h in range(Hkv):
+                for i in range(d):
+                    want_k[dt[s][j // 5], h, j % 5, i] = sk[st[s][j // 3], h, j % 3, i]
+                    want_v[dt[s][j // 5], h, j % 5, i] = sv[st[s][j // 3], h, j % 3, i]
+    np.testing.assert_array_equal(dk, want_k)
+    np.testing.assert_array_equal(dv, want_v)
+
+
+def pin_copy_state_round_trip(lib=None):
+    # pages of 4 -> a linear buffer (one page of 16 per stream) -> pages of 7
+    rng = np.random.default_rng(20)
+    Hkv, d = 3, 4
+    lens = np.array([13, 16, 1], dtype=np.int32)
+    sk, sv = _state_pool(rng, 14, Hkv, 4, d)
+    st = rng.permutation(14)[:12].reshape(3, 4).astype(np.int32)
+    lk, lv = _state_pool(rng, 3, Hkv, 16, d, fill=synth.BF16_NAN)
+    lt = np.array([[2], [0], [1]], dtype=np.int32)
+    oracle.copy_state(sk, sv, st, lk, lv, lt, lens, lib=lib)
+    for s in range(3):
+        n = int(lens[s])
+        np.testing.assert_array_equal(lk[lt[s][0], :, :n].transpose(1, 0, 2),
+                                      _gather_linear(sk, st[s], n))
+        np.testing.assert_array_equal(lv[lt[s][0], :, :n].transpose(1, 0, 2),
+                                      _gather_linear(sv, st[s], n))
+        assert (lk[lt[s][0], :, n:] == synth.BF16_NAN).all()
+    dk, dv = _state_pool(rng, 10, Hkv, 7, d, fill=synth.BF16_NAN)
+    dt = rng.permutation(10)[:9].reshape(3, 3).astype(np.int32)
+    oracle.copy_state(lk, lv, lt, dk, dv, dt, lens, lib=lib)
+    for s in range(3):
+        n = int(lens[s])
+        np.testing.assert_array_equal(_gather_linear(dk, dt[s], n), _gather_linear(sk, st[s], n))
+        np.testing.assert_array_equal(_gather_linear(dv, dt[s], n), _gather_linear(sv, st[s], n))
+
+
+def pin_copy_state_matches_put_rows(lib=None):
+    # resuming a linear state into pages is the row write of all its rows
+    rng = np.random.default_rng(21)
+    Hkv, d, P = 2, 5, 3
+    lens = np.array([8, 8], dtype=np.int32)
+    lk, lv = _state_pool(rng, 2, Hkv, 8, d)
+    lt = np.array([[1], [0]], dtype=np.int32)
+    dt = np.array([[5, 0, 3], [2, 6, 4]], dtype=np.int32)
+    ak, av = _state_pool(rng, 7, Hkv, P, d, fill=synth.BF16_NAN)
+    oracle.copy_state(lk, lv, lt, ak, av, dt, lens, lib=lib)
+    bk, bv = _state_pool(rng, 7, Hkv, P, d, fill=synth.BF16_NAN)
+    rows_k = np.stack([lk[lt[s][0]].transpose(1, 0, 2) for s in range(2)])   # [S][8][Hkv][d]
+    rows_v = np.stack([lv[lt[s][0]].transpose(1, 0, 2) for s in range(2)])
+    oracle.put_rows(bk, bv, dt, lens, rows_k, rows_v, lib=lib)
+    np.testing.assert_array_equal(ak, bk)
+    np.testing.assert_array_equal(av, bv)
+
+
 ALL_PINS = [pin_hand_examples, pin_brute_force, pin_sdpa, pin_closed_forms, pin_invariants,
-            pin_put_rows, pin_tree_brute_force, pin_tree_sdpa, pin_tree_paths]
+            pin_put_rows, pin_tree_brute_force, pin_tree_sdpa, pin_tree_paths,
+            pin_copy_state_brute, pin_copy_state_round_trip, pin_copy_state_matches_put_rows]

@@ -33,6 +33,14 @@ PLANTS = [
      "return (J->tree[(int64_t)s * J->W + (J->W - 1 - r)] >> (j - base)) & 1;"),
     ("tree mask shifted by one key", "return (J->tree[(int64_t)s * J->W + r] >> (j - base)) & 1;",
      "return (J->tree[(int64_t)s * J->W + r] >> (j - base + 1)) & 1;"),
+    ("copy destination slot off by one",
+     "const int64_t to = (((int64_t)dp * Hkv + kh) * dst_P + j % dst_P) * d;",
+     "const int64_t to = (((int64_t)dp * Hkv + kh) * dst_P + (j + 1) % dst_P) * d;"),
+    ("copy drops the last position", "for (j = 0; j < lens[s]; ++j) {\n            const int32_t sp",
+     "for (j = 0; j + 1 < lens[s]; ++j) {\n            const int32_t sp"),
+    ("copy reads the mirrored KV head",
+     "const int64_t from = (((int64_t)sp * Hkv + kh) * src_P + j % src_P) * d;",
+     "const int64_t from = (((int64_t)sp * Hkv + (Hkv - 1 - kh)) * src_P + j % src_P) * d;"),
     ("row write slot off by one", "const int64_t slot = pos % P;",
      "const int64_t slot = (pos + 1) % P;"),
     ("row write pool index transposed", "(((int64_t)page * Hkv + kh) * P + slot) * d;",
