@@ -36,6 +36,7 @@ causal TFLOP/s) and the shape variants ("variants": GQA 12, GQA 16 at head dim
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -141,6 +142,65 @@ def measure_other(name, args, barrier, dist, world, local):
     if 1 < wl.w.rows <= 8:
         out["verify_tokens_per_s"] = out["rows_per_s"]
     del wl
+    return out
+
+
+def measure_state_copy(args, barrier, dist, world, local):
+    """The page-walking state copy (tf_kv_copy_state) of the decode workload's
+    state: 12 streams x 40,960 positions x 8 KV heads at head dim 128, from its
+    shuffled pages to another shuffled set of pages in a second pool.  Bytes
+    are read + write (the measured copy peak counts the same way)."""
+    import torch
+    import synth
+    wl = Workload("decode_12x40k", f"cuda:{local}")
+    tf, w = wl.tf, wl.w
+    w2 = dataclasses.replace(w, seed=w.seed + 1000)
+    t2, n2, _ = synth.page_table(w2, wl.lens_np)
+    dst_table = torch.from_numpy(t2).to(wl.k_pool.device)
+    shape = (n2, w.n_kv_heads, w.page_size, w.head_dim)
+    dk = torch.empty(shape, dtype=torch.bfloat16, device=wl.k_pool.device)
+    dv = torch.empty(shape, dtype=torch.bfloat16, device=wl.k_pool.device)
+    status = torch.zeros(1, dtype=torch.int32, device=wl.k_pool.device)
+
+    def copy():
+        tf.tf_kv_copy_state(wl.k_pool, wl.v_pool, wl.table, wl.lens, dk, dv, dst_table,
+                            wl.max_len, status=status)
+    for _ in range(args.warmup):
+        copy()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for e0, e1 in ev:
+        e0.record()
+        copy()
+        e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"state copy status {int(status.item()):#x}")
+    # every copied byte checked once, after timing: the destination holds the source's rows
+    ok = all(torch.equal(dk[t2[0, i]], wl.k_pool[wl.table[0, i]]) for i in (0, 7, 79))
+    moved = 2 * kv_bytes(wl.lens_np, w.n_kv_heads, w.head_dim)      # read + write
+    gbs = world * moved / (ms * 1e-3) / 1e9
+    peak, src = hbm_peak()
+    out = {"workload": "state_copy_12x40k", "value": gbs, "unit": "GB/s", "ms_per_step": ms,
+           "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peak, "unit": "GB/s",
+                        "frac": gbs / world / peak, "traffic": None, "kernel": "kv_copy_kernel",
+                        "peak_source": src},
+           "check": "sampled pages equal" if ok else "MISMATCH",
+           "gpu_launches": args.steps,
+           "config": {"workload": "state_copy_12x40k", "streams": 12, "context": 40960,
+                      "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "page_size": w.page_size,
+                      "bytes": "K+V read and written", "parallelism": "replicas",
+                      "l2": f"inputs {moved / 2e9:.2f} GB > 126 MB L2"}}
+    del wl, dk, dv
+    torch.cuda.empty_cache()
     return out
 
 
@@ -602,6 +662,7 @@ def main():
                      "decode_12x40k_p37"):
             line["variants"].append(measure_other(name, args, barrier, dist, world, local))
             torch.cuda.empty_cache()
+        line["state_copy"] = measure_state_copy(args, barrier, dist, world, local)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import synth

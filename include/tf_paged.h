@@ -123,6 +123,30 @@ TF_API int tf_kv_put_rows(const tf_kv_pool *pool, const tf_streams *streams,
                    const void *k_rows, const void *v_rows, int32_t rows,
                    void *stream);
 
+/* The state copy (TensorFold #1620, opening comment, "Kept states" bullet:
+ * a kept state is copied by walking the slot's pages).  For every stream s
+ * and position j < src->lens[s], the head_dim bf16 values of K and of V of
+ * every KV head are copied bit for bit from src_pool page
+ * src->table[s][j / src page_size], slot j % src page_size, to dst_pool page
+ * dst_table[s][j / dst page_size], slot j % dst page_size.  Nothing else of
+ * dst_pool is written.  The pools may be the same or differ in n_pages and
+ * page_size; n_kv_heads and head_dim must match.  A linear buffer is a pool
+ * with one page per stream (page_size >= the state's length), so keeping a
+ * state (pages to linear), resuming it (linear to pages) and moving it
+ * between pages are all this call.
+ *  src, src_pool  as for the attention calls (src->max_len bounds every
+ *                 lens[s] and sizes the launch)
+ *  dst_table      device int32 [n_streams][dst_table_stride], caller-owned;
+ *                 dst_table_stride * dst page_size must be >= src->max_len
+ *  status         optional device uint32 (4-byte aligned): TF_DEV_BAD_LEN and
+ *                 TF_DEV_BAD_PAGE are ORed in for skipped streams and pieces
+ * The copied source and destination ranges must not overlap.  Returns
+ * TF_OK, TF_EINVAL (bad or mismatched arguments), TF_EUNSUPPORTED (head_dim)
+ * or TF_ECUDA; enqueued on `stream`. */
+TF_API int tf_kv_copy_state(const tf_kv_pool *src_pool, const tf_streams *src,
+                            const tf_kv_pool *dst_pool, const int32_t *dst_table,
+                            int32_t dst_table_stride, uint32_t *status, void *stream);
+
 /* Workspace bytes an attention call with these arguments needs on the
  * current device (0 on a bad argument), for any of the attention calls
  * with these arguments (tf_paged_attn_verify_tree included).  The workspace holds split-context

@@ -100,3 +100,20 @@ def test_tree_verify_host_checks(lib):
     # more rows than a mask byte holds
     assert lib.raw.tf_paged_attn_verify_tree(ctypes.byref(pool), ctypes.byref(st), 16, 8, 9, 16,
                                              0.1, 16, 16, 1 << 30, None) == lib.TF_EINVAL
+
+
+def test_copy_state_host_checks(lib):
+    src, st = _pool(lib), _streams(lib)
+    dst = _pool(lib, page_size=37)
+    # mismatched head dim or KV heads
+    for bad in (_pool(lib, head_dim=512), _pool(lib, n_kv_heads=3)):
+        assert lib.raw.tf_kv_copy_state(ctypes.byref(src), ctypes.byref(st), ctypes.byref(bad), 16,
+                                        64, None, None) == lib.TF_EINVAL
+    # destination table too short for max_len (2048 > 50 * 37)
+    assert lib.raw.tf_kv_copy_state(ctypes.byref(src), ctypes.byref(st), ctypes.byref(dst), 16, 50,
+                                    None, None) == lib.TF_EINVAL
+    # no destination table, an unaligned status word
+    assert lib.raw.tf_kv_copy_state(ctypes.byref(src), ctypes.byref(st), ctypes.byref(dst), None,
+                                    64, None, None) == lib.TF_EINVAL
+    assert lib.raw.tf_kv_copy_state(ctypes.byref(src), ctypes.byref(st), ctypes.byref(dst), 16, 64,
+                                    18, None) == lib.TF_EINVAL

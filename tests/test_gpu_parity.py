@@ -413,3 +413,90 @@ def test_page37_bad_page_is_flagged_and_shapes_refused():
     with pytest.raises(tf.TFError) as e:
         dc3.attend(ws=ws2, q=dc3.q, tree=synth.tree_masks((11302,), 1, 4))
     assert e.value.status == tf.TF_EUNSUPPORTED
+
+
+# --- the state copy: a stream's K/V walked from one set of pages to another
+
+def _u16(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("sP,dP", [(512, 512), (512, 37), (37, 64), (64, 1), (1, 512), (128, 100)])
+@pytest.mark.parametrize("d", [128, 512])
+def test_copy_state_bit_exact(sP, dP, d):
+    import verify_paged_gqa_b200 as tf
+    rng = np.random.default_rng(12000 + sP + dP + d)
+    Hkv = 2
+    lens = np.array([700, 0, 1, 1537], dtype=np.int32)
+    ws = synth.Workload("copy", 4, Hkv, 4, d, sP, 1, seed=12001 + sP)
+    wd = synth.Workload("copy", 4, Hkv, 4, d, dP, 1, seed=12002 + dP)
+    st, sn, _ = synth.page_table(ws, np.maximum(lens, 1))
+    dt, dn, _ = synth.page_table(wd, np.maximum(lens, 1))
+    sk = rng.integers(0, 0xFFFF, size=(sn, Hkv, sP, d)).astype(np.uint16)
+    sv = rng.integers(0, 0xFFFF, size=(sn, Hkv, sP, d)).astype(np.uint16)
+    dk = np.full((dn, Hkv, dP, d), synth.BF16_NAN, dtype=np.uint16)
+    dv = dk.copy()
+    gk, gv = bf16_tensor(dk), bf16_tensor(dv)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tf.tf_kv_copy_state(bf16_tensor(sk), bf16_tensor(sv), torch.from_numpy(st).cuda(),
+                        torch.from_numpy(lens).cuda(), gk, gv, torch.from_numpy(dt).cuda(),
+                        max_len=int(lens.max()), status=status)
+    oracle.copy_state(sk, sv, st, dk, dv, dt, lens)
+    assert np.array_equal(_u16(gk), dk)
+    assert np.array_equal(_u16(gv), dv)
+    assert int(status.item()) == 0
+
+
+def test_copy_state_keep_and_resume_give_the_same_attention():
+    """Keep every stream's state in a linear buffer (one page per stream), resume
+    it into other shuffled pages of the same pool's spare room, and attend: the
+    output is byte-equal to attending over the original pages."""
+    import verify_paged_gqa_b200 as tf
+    W = 4
+    w = small_workload(128, 8, 512, W, seed=12100)
+    lens = [3000, 513, 2048]
+    case = synth.make_case(w, lens=lens)
+    a_dc = DeviceCase(case)
+    a = a_dc.attend()
+    L = int(max(lens))
+    lin_k = torch.full((3, 2, L, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lin_v = lin_k.clone()
+    lin_t = torch.arange(3, dtype=torch.int32, device="cuda")[:, None].contiguous()
+    tf.tf_kv_copy_state(a_dc.k_pool, a_dc.v_pool, a_dc.table, a_dc.lens, lin_k, lin_v, lin_t,
+                        max_len=L)
+    # the linear state holds the stream's rows in order
+    for s in range(3):
+        n = lens[s]
+        assert np.array_equal(_u16(lin_k[s, :, :n].transpose(0, 1).contiguous()), case.k_lin[s])
+    w2 = synth.Workload("sweep", 0, 2, 8, 128, 512, W, seed=12101)
+    t2, n2, _ = synth.page_table(w2, case.lens)
+    b_dc = DeviceCase(case, table=t2, n_pages=n2)
+    b_dc.k_pool.fill_(float("nan"))
+    b_dc.v_pool.fill_(float("nan"))
+    tf.tf_kv_copy_state(lin_k, lin_v, lin_t, a_dc.lens, b_dc.k_pool, b_dc.v_pool, b_dc.table,
+                        max_len=L)
+    b = b_dc.attend()
+    assert torch.equal(a, b)
+
+
+def test_copy_state_flags_bad_pages_and_lengths():
+    import verify_paged_gqa_b200 as tf
+    Hkv, d, P = 2, 128, 64
+    sk = torch.randn(6, Hkv, P, d, device="cuda").to(torch.bfloat16)
+    sv = torch.randn(6, Hkv, P, d, device="cuda").to(torch.bfloat16)
+    dk = torch.zeros(6, Hkv, P, d, dtype=torch.bfloat16, device="cuda")
+    dv = dk.clone()
+    st = torch.tensor([[0, 1, 2], [3, 4, 5]], dtype=torch.int32, device="cuda")
+    dt = torch.tensor([[5, 4, 3], [2, 1, 99]], dtype=torch.int32, device="cuda")  # 99: bad
+    lens = torch.tensor([150, 140], dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tf.tf_kv_copy_state(sk, sv, st, lens, dk, dv, dt, max_len=192, status=status)
+    assert int(status.item()) & tf.TF_DEV_BAD_PAGE
+    # stream 0 was copied whole; stream 1's good pages too
+    assert torch.equal(dk[5], sk[0]) and torch.equal(dk[4], sk[1])
+    assert torch.equal(dk[3, :, :150 - 128], sk[2, :, :150 - 128])
+    assert torch.equal(dv[2], sv[3]) and torch.equal(dv[1], sv[4])
+    status.zero_()
+    lens2 = torch.tensor([150, 300], dtype=torch.int32, device="cuda")   # past max_len
+    tf.tf_kv_copy_state(sk, sv, st, lens2, dk, dv, st, max_len=192, status=status)
+    assert int(status.item()) & tf.TF_DEV_BAD_LEN

@@ -10,7 +10,7 @@ imports without it.
 _EXPORTS = (
     "TF_DEV_BAD_LEN", "TF_DEV_BAD_PAGE", "TF_DEV_TIMEOUT", "TF_EINVAL", "TF_ENOSPACE",
     "TF_ECUDA", "TF_EUNSUPPORTED", "TF_OK", "TFError", "library_path", "raw",
-    "tf_kv_put_rows", "tf_paged_attn_decode", "tf_paged_attn_prompt", "tf_paged_attn_verify",
+    "tf_kv_copy_state", "tf_kv_put_rows", "tf_paged_attn_decode", "tf_paged_attn_prompt", "tf_paged_attn_verify",
     "tf_paged_attn_verify_tree", "tf_paged_attn_workspace_bytes", "tf_status_str",
     "tf_workspace_status",
 )

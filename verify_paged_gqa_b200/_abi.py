@@ -82,6 +82,9 @@ for _name in ("tf_paged_attn_verify", "tf_paged_attn_prompt"):
 raw.tf_paged_attn_verify_tree.argtypes = [_P(tf_kv_pool), _P(tf_streams), _vp, _i32, _i32, _vp,
                                           _f32, _vp, _vp, _sz, _vp]
 raw.tf_paged_attn_verify_tree.restype = ctypes.c_int
+raw.tf_kv_copy_state.argtypes = [_P(tf_kv_pool), _P(tf_streams), _P(tf_kv_pool), _vp, _i32, _vp,
+                                 _vp]
+raw.tf_kv_copy_state.restype = ctypes.c_int
 raw.tf_workspace_status.argtypes = [_vp, _P(ctypes.c_uint32), _vp]
 raw.tf_workspace_status.restype = ctypes.c_int
 raw.tf_status_str.argtypes = [ctypes.c_int]
@@ -143,6 +146,27 @@ def tf_kv_put_rows(k_pool, v_pool, table, lens, k_rows, v_rows, max_len, stream=
     _check(raw.tf_kv_put_rows(ctypes.byref(pool), ctypes.byref(st), k_rows.data_ptr(),
                               v_rows.data_ptr(), k_rows.shape[1], _stream(stream)),
            "tf_kv_put_rows")
+
+
+def tf_kv_copy_state(src_k, src_v, src_table, lens, dst_k, dst_v, dst_table, max_len,
+                     status=None, stream=None):
+    """Copies every stream's positions [0, lens[s]) of K and V from the source
+    pools' pages (src_table) to the destination pools' pages (dst_table).
+    status: optional uint32-viewable int32 device tensor of one element that
+    collects TF_DEV_* bits."""
+    src_pool, st = _pool(src_k, src_v), _streams(src_table, lens, max_len)
+    dst_pool = _pool(dst_k, dst_v)
+    _need(dst_table, torch.int32, 2, "dst_table")
+    if dst_table.shape[0] != lens.shape[0]:
+        raise ValueError("dst_table must have one row per stream")
+    sp = 0
+    if status is not None:
+        if status.dtype != torch.int32 or status.numel() < 1:
+            raise TypeError("status must be an int32 tensor")
+        sp = status.data_ptr()
+    _check(raw.tf_kv_copy_state(ctypes.byref(src_pool), ctypes.byref(st), ctypes.byref(dst_pool),
+                                dst_table.data_ptr(), dst_table.shape[1], sp or None,
+                                _stream(stream)), "tf_kv_copy_state")
 
 
 def tf_paged_attn_workspace_bytes(k_pool, v_pool, table, lens, n_q_heads, rows, max_len) -> int:

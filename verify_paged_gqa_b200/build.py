@@ -19,7 +19,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build", "tfpaged")
 LIB = os.path.join(HERE, "libtfpaged.so")
-SOURCES = ["tf_paged.cu", "kv_put.cu", "attn_simt.cu", "attn_prompt.cu", "attn_pm.cu", "attn_merge.cu"]
+SOURCES = ["tf_paged.cu", "kv_put.cu", "kv_copy.cu", "attn_simt.cu", "attn_prompt.cu", "attn_pm.cu",
+           "attn_merge.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr",
          "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]

@@ -18,6 +18,26 @@ struct PutParams {
 
 cudaError_t launch_kv_put(const PutParams &p, cudaStream_t stream);
 
+// The state copy (kv_copy.cu): positions [0, lens[s]) of every KV head from
+// the source pool's pages to the destination pool's pages.
+struct CopyParams {
+    const __nv_bfloat16 *src_k;
+    const __nv_bfloat16 *src_v;
+    __nv_bfloat16 *dst_k;
+    __nv_bfloat16 *dst_v;
+    const int32_t *src_table;
+    const int32_t *dst_table;
+    const int32_t *lens;
+    uint32_t *status;              // TF_DEV_* bits are ORed in (may be null)
+    int32_t src_stride, dst_stride, src_P, dst_P, src_n_pages, dst_n_pages;
+    int32_t Hkv, D, S, max_len;
+    int32_t chunk;                 // positions per block
+    int32_t n_chunks;              // blocks per (stream, KV head): ceil(max_len / chunk)
+};
+
+int copy_chunk_positions(int head_dim);
+cudaError_t launch_kv_copy(const CopyParams &p, cudaStream_t stream);
+
 // Rows per row block of the CUDA-core partial kernel.
 constexpr int kSimtRows = 4;
 

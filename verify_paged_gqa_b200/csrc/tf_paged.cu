@@ -262,6 +262,54 @@ int tf_kv_put_rows(const tf_kv_pool *pool, const tf_streams *streams, const void
     return launch_kv_put(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_ECUDA;
 }
 
+int tf_kv_copy_state(const tf_kv_pool *src_pool, const tf_streams *src,
+                     const tf_kv_pool *dst_pool, const int32_t *dst_table,
+                     int32_t dst_table_stride, uint32_t *status, void *stream)
+{
+    int rc = check_pool_streams(src_pool, src);
+    if (rc != TF_OK)
+        return rc;
+    if (!dst_pool || dst_pool->n_pages < 1 || dst_pool->page_size < 1)
+        return TF_EINVAL;
+    if (dst_pool->n_kv_heads != src_pool->n_kv_heads || dst_pool->head_dim != src_pool->head_dim)
+        return TF_EINVAL;
+    if (!dst_pool->k_pool || !dst_pool->v_pool || !aligned16(dst_pool->k_pool) ||
+        !aligned16(dst_pool->v_pool))
+        return TF_EINVAL;
+    if (dst_table_stride < 1 ||
+        (int64_t)src->max_len > (int64_t)dst_table_stride * dst_pool->page_size ||
+        (int64_t)src->n_streams * dst_table_stride > INT32_MAX)
+        return TF_EINVAL;
+    if (src->n_streams > 0 && !dst_table)
+        return TF_EINVAL;
+    if (status && (reinterpret_cast<uintptr_t>(status) & 3u) != 0)
+        return TF_EINVAL;
+    if (src->n_streams == 0)
+        return TF_OK;
+    CopyParams p;
+    p.src_k = static_cast<const __nv_bfloat16 *>(src_pool->k_pool);
+    p.src_v = static_cast<const __nv_bfloat16 *>(src_pool->v_pool);
+    p.dst_k = static_cast<__nv_bfloat16 *>(dst_pool->k_pool);
+    p.dst_v = static_cast<__nv_bfloat16 *>(dst_pool->v_pool);
+    p.src_table = src->table;
+    p.dst_table = dst_table;
+    p.lens = src->lens;
+    p.status = status;
+    p.src_stride = src->table_stride;
+    p.dst_stride = dst_table_stride;
+    p.src_P = src_pool->page_size;
+    p.dst_P = dst_pool->page_size;
+    p.src_n_pages = src_pool->n_pages;
+    p.dst_n_pages = dst_pool->n_pages;
+    p.Hkv = src_pool->n_kv_heads;
+    p.D = src_pool->head_dim;
+    p.S = src->n_streams;
+    p.max_len = src->max_len;
+    p.chunk = copy_chunk_positions(p.D);
+    p.n_chunks = (src->max_len + p.chunk - 1) / p.chunk;
+    return launch_kv_copy(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TF_OK : TF_ECUDA;
+}
+
 size_t tf_paged_attn_workspace_bytes(const tf_kv_pool *pool, const tf_streams *streams,
                                      int32_t n_q_heads, int32_t rows)
 {
