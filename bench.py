@@ -145,14 +145,15 @@ def measure_other(name, args, barrier, dist, world, local):
     return out
 
 
-def measure_state_copy(args, barrier, dist, world, local):
-    """The page-walking state copy (tf_kv_copy_state) of the decode workload's
-    state: 12 streams x 40,960 positions x 8 KV heads at head dim 128, from its
-    shuffled pages to another shuffled set of pages in a second pool.  Bytes
-    are read + write (the measured copy peak counts the same way)."""
+def measure_state_copy(args, barrier, dist, world, local, name="decode_12x40k"):
+    """The page-walking state copy (tf_kv_copy_state) of a workload's state (by
+    default the decode workload's: 12 streams x 40,960 positions x 8 KV heads
+    at head dim 128), from its shuffled pages to another shuffled set of pages
+    in a second pool.  Bytes are read + write (the measured copy peak counts
+    the same way)."""
     import torch
     import synth
-    wl = Workload("decode_12x40k", f"cuda:{local}")
+    wl = Workload(name, f"cuda:{local}")
     tf, w = wl.tf, wl.w
     w2 = dataclasses.replace(w, seed=w.seed + 1000)
     t2, n2, _ = synth.page_table(w2, wl.lens_np)
@@ -185,17 +186,20 @@ def measure_state_copy(args, barrier, dist, world, local):
     if int(status.item()) != 0:
         raise RuntimeError(f"state copy status {int(status.item()):#x}")
     # every copied byte checked once, after timing: the destination holds the source's rows
-    ok = all(torch.equal(dk[t2[0, i]], wl.k_pool[wl.table[0, i]]) for i in (0, 7, 79))
+    n_full = int(wl.lens_np[0]) // w.page_size      # stream 0's full pages
+    ok = all(torch.equal(dk[t2[0, i]], wl.k_pool[wl.table[0, i]])
+             for i in sorted({0, n_full // 2, n_full - 1}) if n_full > 0)
     moved = 2 * kv_bytes(wl.lens_np, w.n_kv_heads, w.head_dim)      # read + write
     gbs = world * moved / (ms * 1e-3) / 1e9
     peak, src = hbm_peak()
-    out = {"workload": "state_copy_12x40k", "value": gbs, "unit": "GB/s", "ms_per_step": ms,
+    label = "state_copy_" + name.split("_", 1)[1] if "_" in name else "state_copy_" + name
+    out = {"workload": label, "value": gbs, "unit": "GB/s", "ms_per_step": ms,
            "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peak, "unit": "GB/s",
                         "frac": gbs / world / peak, "traffic": None, "kernel": "kv_copy_kernel",
                         "peak_source": src},
            "check": "sampled pages equal" if ok else "MISMATCH",
            "gpu_launches": args.steps,
-           "config": {"workload": "state_copy_12x40k", "streams": 12, "context": 40960,
+           "config": {"workload": label, "streams": len(wl.lens_np), "context": int(wl.lens_np.max()),
                       "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "page_size": w.page_size,
                       "bytes": "K+V read and written", "parallelism": "replicas",
                       "l2": f"inputs {moved / 2e9:.2f} GB > 126 MB L2"}}
@@ -591,6 +595,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-verify", action="store_true", help="skip the verify-workload measurement")
+    ap.add_argument("--state-copy", action="store_true",
+                    help="time only the state copy (tf_kv_copy_state) of --workload's state")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -611,6 +617,14 @@ def main():
     def barrier():
         if dist is not None:
             dist.barrier()
+
+    if args.state_copy:
+        out = measure_state_copy(args, barrier, dist, world, local, name=args.workload)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
 
     wl = Workload(args.workload, f"cuda:{local}")
     uuid = str(torch.cuda.get_device_properties(local).uuid)
