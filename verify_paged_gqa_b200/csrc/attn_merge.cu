@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
     const int nseg = nseg_sh;
     if (nseg == 0)
         return;
-    const size_t slot_floats = (size_t)p.SR * (D + 2);
+    const size_t slot_floats = part_slot_floats(p);
 
     for (int m = m0 + warp; m < m1; m += nwarps) {
         const int r = m - mb;

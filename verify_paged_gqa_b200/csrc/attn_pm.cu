@@ -564,7 +564,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
         named_barrier(1, NT);
         const bool write = ok && !sm.abort_flag;
         float *slot = fin ? nullptr
-                          : p.part + (size_t)it.slot * (p.SR * (D + 2));
+                          : p.part + (size_t)it.slot * part_slot_floats(p);
 #pragma unroll 1
         for (int vb = 0; vb < C::DB; ++vb) {
             uint32_t hi[32], lo[32];

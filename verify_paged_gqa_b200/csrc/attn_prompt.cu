@@ -383,7 +383,7 @@ __device__ __forceinline__ void pr_softmax(const PrArgs &a, PrSmem &sm, int warp
         sm.lhalf[hh][r] = lacc.x + lacc.y;
         named_barrier(1, 256);
         const bool write = ok && !sm.abort_flag;
-        float *slot = it.fin ? nullptr : p.part + (size_t)it.slot * (p.SR * (DD + 2));
+        float *slot = it.fin ? nullptr : p.part + (size_t)it.slot * part_slot_floats(p);
         // O^T lane r is head dim r; this thread takes rows [64 hh, 64 hh + 64)
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {

@@ -620,7 +620,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 scale_out = 1.f / lstar;
             } else {
                 float *slot =
-                    p.part + (size_t)it.slot * (p.SR * (D + 2));
+                    p.part + (size_t)it.slot * part_slot_floats(p);
                 dst = slot + (size_t)r * D;
                 scale_out = 1.f;
                 if (lane == 0) {

@@ -59,6 +59,14 @@ struct AttnParams {
     float scale_log2;           // scale * log2(e): scores are kept in log2 units
 };
 
+// Floats per partial slot: SR rows of O (D floats each), then SR running
+// maxima and SR running sums, rounded up to 16 bytes so every slot (and every
+// row of O in it) starts 16-byte aligned.
+__host__ __device__ __forceinline__ size_t part_slot_floats(const AttnParams &p)
+{
+    return ((size_t)p.SR * (p.D + 2) + 3) & ~(size_t)3;
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -151,6 +159,29 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
 }
+
+// Bulk copy (TMA engine) of `bytes` from this CTA's shared memory to global
+// memory, in the issuing thread's current bulk group.  Both addresses 16-byte
+// aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(static_cast<uint32_t>(__cvta_generic_to_shared(src))), "r"(bytes)
+                 : "memory");
+}
+
+// Closes the issuing thread's current bulk group.
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Waits until at most N of the thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Waits until all of the thread's bulk groups are complete (writes performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // L2 policy for data read once per call (K/V streams): evict first.
 __device__ __forceinline__ uint64_t l2_evict_first_policy()

@@ -58,7 +58,7 @@ enum class Kernel { kSimt, kPrompt, kPm };
 
 // Workspace: the 256-byte header (status word, wait site, the launch's tile
 // count at byte 64), each stream's first tile (int64), then two partial slots
-// per CTA of min(RB, M) rows x (D + 2) floats.
+// per CTA of min(RB, M) rows x (D + 2) floats (rounded up to 16 bytes).
 constexpr size_t kWsTotalOffset = 64;
 
 size_t ws_part_offset(int S)
@@ -168,7 +168,7 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
         grid = units > 0 ? units : 1;
     plan->grid = static_cast<int>(grid);
     p.n_cta = plan->grid;
-    plan->ws_bytes = ws_part_offset(p.S) + (size_t)2 * plan->grid * p.SR * (p.D + 2) * sizeof(float);
+    plan->ws_bytes = ws_part_offset(p.S) + (size_t)2 * plan->grid * part_slot_floats(p) * sizeof(float);
     return TF_OK;
 }
 
