@@ -71,7 +71,7 @@ size_t ws_part_offset(int S)
 // tile, so the pipeline drains and refills); the CUDA-core decode kernel's
 // segment starts overlap with its deep ring and cost nothing measurable.
 constexpr int kEntryPm512 = 8;
-constexpr int kEntryPm128 = 4;
+constexpr int kEntryPm128 = 6;
 constexpr int kEntryPrompt = 4;
 constexpr int kEntrySimt = 0;
 
