@@ -93,8 +93,8 @@ extern "C" {
  * contract bullet: the paged prompt kernel is checked over pages of 512, 37
  * and 64); head_dim must be 128, 256 or 512.  The tensor-core kernels need
  * page_size a multiple of 128: other sizes run on the CUDA-core kernel,
- * whose tiles may then straddle pages, and head dim 256 and tree-mask calls
- * are refused for them (TF_EUNSUPPORTED). */
+ * whose tiles may then straddle pages, and head dim 256 calls are refused
+ * for them (TF_EUNSUPPORTED). */
 typedef struct tf_kv_pool {
     void *k_pool;
     void *v_pool;
@@ -189,7 +189,8 @@ TF_API int tf_paged_attn_verify(const tf_kv_pool *pool, const tf_streams *stream
  *              (no context before the window and an empty mask) gets NaN.
  * Everything else (arguments, layouts, results, the workspace, errors) is
  * as tf_paged_attn_verify; TF_EINVAL also when tree_masks is null, and
- * TF_EUNSUPPORTED when page_size is not a multiple of 128.  Head dim 128
+ * TF_EUNSUPPORTED for head dim 256 with a page_size that is not a multiple
+ * of 128.  Head dim 128
  * calls with more than 64 query rows per KV head (G * rows) read each K/V
  * tile once per 64 rows. */
 TF_API int tf_paged_attn_verify_tree(const tf_kv_pool *pool, const tf_streams *streams,

@@ -336,15 +336,13 @@ def test_tree_growing_scores():
     assert max_abs(out, ref) <= TOL
 
 
-def test_tree_needs_pages_of_128():
-    import verify_paged_gqa_b200 as tf
-    w = small_workload(128, 4, 64, 4, seed=10600)
-    case = synth.make_case(w, lens=[300], rows=4)
-    dc = DeviceCase(case)
-    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
-    with pytest.raises(tf.TFError) as e:
-        dc.attend(ws=ws, tree=synth.tree_masks((10601,), 1, 4))
-    assert e.value.status == tf.TF_EUNSUPPORTED
+@pytest.mark.parametrize("P", [64, 37])
+@pytest.mark.parametrize("d,G,W", [(128, 4, 4), (128, 8, 8), (512, 8, 3)])
+def test_tree_any_page_size(P, d, G, W):
+    """Pages that are not a multiple of 128 take tree calls on the CUDA-core kernel."""
+    w = small_workload(d, G, P, W, seed=10600 + P + d + G + W)
+    lens = [P * 5 + 3, W, 700]
+    run_tree_parity(w, lens, W, synth.tree_masks((10601, P, d, G, W), len(lens), W))
 
 
 # --- any page size (the pages check the paged prompt kernel over pages of 37):
@@ -402,17 +400,14 @@ def test_page37_bad_page_is_flagged_and_shapes_refused():
     dc.table[0, 3] = dc.k_pool.shape[0] + 2      # a page in the middle of a straddling tile
     dc.attend(ws=ws)
     assert tf.tf_workspace_status(ws) & tf.TF_DEV_BAD_PAGE
-    # head dim 256 and tree masks need pages that are a multiple of 128
+    # head dim 256 (with or without tree masks) needs pages that are a multiple of 128
     w2 = small_workload(256, 4, 37, 4, seed=11301)
     dc2 = DeviceCase(synth.make_case(w2, lens=[300], rows=4))
     ws2 = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
-    with pytest.raises(tf.TFError) as e:
-        dc2.attend(ws=ws2)
-    assert e.value.status == tf.TF_EUNSUPPORTED
-    dc3 = DeviceCase(synth.make_case(w, lens=[300], rows=4))
-    with pytest.raises(tf.TFError) as e:
-        dc3.attend(ws=ws2, q=dc3.q, tree=synth.tree_masks((11302,), 1, 4))
-    assert e.value.status == tf.TF_EUNSUPPORTED
+    for tree in (None, synth.tree_masks((11302,), 1, 4)):
+        with pytest.raises(tf.TFError) as e:
+            dc2.attend(ws=ws2, tree=tree)
+        assert e.value.status == tf.TF_EUNSUPPORTED
 
 
 # --- the state copy: a stream's K/V walked from one set of pages to another

@@ -314,7 +314,18 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
     }
 }
 
-template <int D>
+// Tree masks (kTree): row r sees the positions before the window (pos <
+// lim[r] = len - W) and window row c when bit c of tm[r] is set.
+template <bool kTree>
+__device__ __forceinline__ bool simt_sees(int pos, int lim, uint32_t tm, int base, int W)
+{
+    if constexpr (kTree)
+        return pos < lim || ((unsigned)(pos - base) < (unsigned)W && ((tm >> (pos - base)) & 1u));
+    else
+        return pos < lim;
+}
+
+template <int D, bool kTree>
 __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &sm, int warp,
                                               int lane)
 {
@@ -347,13 +358,21 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
         // --- this segment's query rows: packed bf16 pairs in registers --------
         uint32_t qh[kR][CPL * 4];
         int lim[kR];
+        uint32_t tm[kR];
+        const int base = it.len - p.W;  // the window's first position
         {
             const int slot = j & 1;
             const bool ok = wait_or_abort(sm, &sm.q_full[slot], (j >> 1) & 1u, p.flags, kWaitQFull);
 #pragma unroll
             for (int r = 0; r < kR; ++r) {
                 const int m = it.b * kR + r;
-                lim[r] = row_lim(p, it.len, m);
+                if constexpr (kTree) {
+                    lim[r] = base;
+                    tm[r] = m < p.M ? __ldg(p.tree + (size_t)it.s * p.W + m / p.G) : 0u;
+                } else {
+                    lim[r] = row_lim(p, it.len, m);
+                    tm[r] = 0u;
+                }
                 const bool live = ok && m < p.M;
 #pragma unroll
                 for (int c = 0; c < CPL; ++c) {
@@ -446,7 +465,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 const int pos = tpos + key;
 #pragma unroll
                 for (int r = 0; r < kR; ++r) {
-                    const bool vis = key < nk && pos < lim[r];
+                    const bool vis = key < nk && simt_sees<kTree>(pos, lim[r], tm[r], base, p.W);
                     sc[r] = vis ? acc[r] * p.scale_log2 : NEG_INF;
                     tmax[r] = warp_max(sc[r], 1);
                 }
@@ -455,7 +474,8 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 const int r = li & 3;
                 const int pos = tpos + key;
                 const int my_lim = r == 0 ? lim[0] : r == 1 ? lim[1] : r == 2 ? lim[2] : lim[3];
-                const bool vis = key < nk && pos < my_lim;
+                const uint32_t my_tm = r == 0 ? tm[0] : r == 1 ? tm[1] : r == 2 ? tm[2] : tm[3];
+                const bool vis = key < nk && simt_sees<kTree>(pos, my_lim, my_tm, base, p.W);
                 sc[0] = vis ? acc[0] * p.scale_log2 : NEG_INF;
                 const float rm = warp_max(sc[0], 4);  // over the lanes of this row
 #pragma unroll
@@ -650,7 +670,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
     }
 }
 
-template <int D>
+template <int D, bool kTree>
 __global__ void __launch_bounds__(simt_threads<D>(), 1)
     attn_simt_kernel(const __grid_constant__ AttnParams p)
 {
@@ -681,12 +701,12 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
         if (lane == 0)
             simt_producer<D>(p, sm);
     } else
-        simt_consumer<D>(p, sm, warp, lane);
+        simt_consumer<D, kTree>(p, sm, warp, lane);
 }
 
 // Host-side launcher (same translation unit as the kernel template).
-template <int D>
-cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream)
+template <int D, bool kTree>
+cudaError_t launch_simt(const AttnParams &p, int grid, cudaStream_t stream)
 {
     const size_t smem = simt_smem_bytes<D>();
     static bool configured[kMaxDevices] = {};  // the attribute is set once per device
@@ -697,14 +717,20 @@ cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream)
     if (dev < 0 || dev >= kMaxDevices)
         return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(attn_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(attn_simt_kernel<D, kTree>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
         if (e != cudaSuccess)
             return e;
         configured[dev] = true;
     }
-    attn_simt_kernel<D><<<grid, simt_threads<D>(), smem, stream>>>(p);
+    attn_simt_kernel<D, kTree><<<grid, simt_threads<D>(), smem, stream>>>(p);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_attn_simt(const AttnParams &p, int grid, cudaStream_t stream)
+{
+    return p.has_tree ? launch_simt<D, true>(p, grid, stream) : launch_simt<D, false>(p, grid, stream);
 }
 
 template cudaError_t launch_attn_simt<128>(const AttnParams &, int, cudaStream_t);

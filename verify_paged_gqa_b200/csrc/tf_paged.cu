@@ -122,12 +122,15 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     plan->kernel = Kernel::kSimt;
     p.RB = kSimtRows;
     if (tree) {
-        // tree masks run on the position-major kernel only (any row count)
+        // tree masks: the position-major kernel (any row count), else the
+        // CUDA-core kernel (page sizes that are not a multiple of 128)
         const int nr = pm_rows(p);
-        if (nr == 0)
+        if (nr > 0) {
+            plan->kernel = Kernel::kPm;
+            p.RB = nr;
+        } else if (p.D == 256) {
             return TF_EUNSUPPORTED;
-        plan->kernel = Kernel::kPm;
-        p.RB = nr;
+        }
     } else if (p.D == 256) {
         // head dim 256 runs on the position-major kernel only (any row count)
         const int nr = pm_rows(p);
