@@ -22,7 +22,8 @@
 // sit side by side along N and land in separate O^T columns that the
 // epilogue adds.
 //
-// One persistent CTA per SM, six warps:
+// One persistent CTA per SM; 2 + NR / 8 warps (six for 32-row blocks, ten
+// for 64):
 //   warp 0     producer (one lane): per tile, the K units of the next tile,
 //              then the V units of this one (a unit is 128 positions x 128
 //              dims, two 64-dim TMA boxes with 128-byte swizzle) into a ring;
@@ -30,7 +31,8 @@
 //   warp 1     MMA issuer (one lane): S^T(t+1) = K Q^T before O^T += V^T P^T(t),
 //              so the softmax of one tile overlaps the MMAs of the next.
 //              Owns the tensor-memory allocation.
-//   warps 2-5  softmax, one key position per thread: write the block's query
+//   warps 2-   softmax (NR / 8 warps), one key position per thread (32 rows
+//              of it): write the block's query
 //              rows into the Q tile at each segment's start; per tile, read the
 //              position's scores for all rows, check them against each row's
 //              reference max (a block-wide vote; the reference moves only

@@ -20,7 +20,7 @@
 // epilogue adds.  16 instructions per tile instead of 24 for a row-major PV
 // run once per half.
 //
-// One persistent CTA per SM, six warps:
+// One persistent CTA per SM, ten warps:
 //   warp 0     producer (one lane): the K/V ring (ring.cuh).
 //   warp 1     MMA issuer (one lane): QK(t + 1) before PV(t).  S has one
 //              tensor-memory buffer: QK(t + 1) starts once the softmax has

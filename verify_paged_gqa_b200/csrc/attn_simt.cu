@@ -15,7 +15,9 @@
 //                 double-buffered shared slot and streams K and V tiles of TK
 //                 positions into a ring of NSTAGE stages with bulk copies
 //                 (TMA engine, no tensor map: a tile of one page and KV head
-//                 is one contiguous run).  Page ids are read one page early.
+//                 is one contiguous run; with a page size that is not a
+//                 multiple of TK a tile may straddle pages and takes one copy
+//                 per page piece).  Page ids are read one page early.
 //   other warps   consumers: tile T of the CTA's sequence goes to consumer
 //                 warp T % NCW.  A warp keeps its own online-softmax state
 //                 (running max m, running sum l, unnormalised O) for the four
@@ -36,7 +38,9 @@
 //           key L.
 //   softmax tile max per row by warp shuffles, exp2 of log2-scaled scores;
 //           masked positions are SELECTED to -inf (never multiplied), so NaN
-//           in unused slots cannot leak.
+//           in unused slots cannot leak.  A causal row sees positions below
+//           its limit; under tree masks (kTree) a row sees the positions
+//           before the window and the window rows its mask byte names.
 //   PV      lane L owns dims 4L..4L+3 of the 4 output rows as fp32 pairs and
 //           updates them with packed fp32 FMAs (two per instruction);
 //           probabilities come from a per-warp shared buffer; only positions
