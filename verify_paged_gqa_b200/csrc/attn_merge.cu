@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
     const float NEG_INF = -__int_as_float(0x7f800000);
     // launched as a programmatic dependent of the partial kernel: wait for
     // that grid to complete (and its writes to be visible) before going on
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    wait_prior_grid();
 
     if (!len_ok(p, len)) {
         if (threadIdx.x == 0 && kh == 0 && b == 0 && g == 0)
@@ -222,17 +222,8 @@ cudaError_t launch_attn_merge(const AttnParams &p, cudaStream_t stream)
     const int threads = 32 * min(kMergeRows, p.RB);
     // programmatic dependent launch: the blocks are scheduled while the
     // partial kernel runs out and wait for it in the kernel
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attn_merge_kernel<D>, p);
+    return launch_dependent(attn_merge_kernel<D>, dim3(static_cast<unsigned>(blocks)), dim3(threads),
+                            0, stream, p);
 }
 
 template cudaError_t launch_attn_merge<128>(const AttnParams &, cudaStream_t);

@@ -625,14 +625,15 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0)
-        find_range(a.p, sm.range, lane);
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr(&sm.tmem_base)), "r"(C::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    wait_prior_grid();
+    if (warp == 0)
+        find_range(a.p, sm.range, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -680,8 +681,8 @@ cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
             return e;
         configured[dev] = true;
     }
-    attn_pm_kernel<D, NR, kTree><<<grid, PmCfg<D, NR>::kThreads, bytes, stream>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(attn_pm_kernel<D, NR, kTree>, dim3(grid), dim3(PmCfg<D, NR>::kThreads),
+                            bytes, stream, a);
 }
 
 }  // namespace

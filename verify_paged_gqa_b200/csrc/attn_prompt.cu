@@ -441,14 +441,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
         sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0)
-        find_range(a.p, sm.range, lane);
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr(&sm.tmem_base)), "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    wait_prior_grid();
+    if (warp == 0)
+        find_range(a.p, sm.range, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -505,8 +506,7 @@ cudaError_t launch_attn_prompt(const AttnParams &p, int grid, cudaStream_t strea
             return e;
         configured[dev] = true;
     }
-    attn_prompt_kernel<<<grid, kThreads, kPrSmemBytes, stream>>>(a);
-    return cudaGetLastError();
+    return launch_dependent(attn_prompt_kernel, dim3(grid), dim3(kThreads), kPrSmemBytes, stream, a);
 }
 
 }  // namespace tfp

@@ -698,6 +698,7 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    wait_prior_grid();
     if (warp == SimtCfg<D>::NCW)
         find_range(p, sm.range, lane);
     __syncthreads();
@@ -727,8 +728,8 @@ cudaError_t launch_simt(const AttnParams &p, int grid, cudaStream_t stream)
             return e;
         configured[dev] = true;
     }
-    attn_simt_kernel<D, kTree><<<grid, simt_threads<D>(), smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(attn_simt_kernel<D, kTree>, dim3(grid), dim3(simt_threads<D>()), smem,
+                            stream, p);
 }
 
 template <int D>

@@ -215,6 +215,15 @@ __device__ __forceinline__ void allow_dependent_launch()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Waits until the previous kernel in the stream has completed and its writes
+// are visible, when this grid was launched as its programmatic dependent (a
+// no-op otherwise).  Nothing a previous kernel may have written (lens, tables,
+// pools, queries) is read before it.
+__device__ __forceinline__ void wait_prior_grid()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void set_flag(uint32_t *flags, uint32_t bit)
 {
     atomicOr(flags, bit);

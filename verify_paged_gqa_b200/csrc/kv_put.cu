@@ -12,6 +12,7 @@ namespace tfp {
 
 __global__ void __launch_bounds__(256) kv_put_kernel(const __grid_constant__ PutParams p)
 {
+    allow_dependent_launch();  // the attention kernel after it may be scheduled now
     const int warps = blockDim.x / 32;
     const int64_t row = (int64_t)blockIdx.x * warps + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;

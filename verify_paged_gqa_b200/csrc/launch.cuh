@@ -5,6 +5,26 @@
 
 namespace tfp {
 
+// Launches `kernel` as a programmatic dependent of the previous kernel in the
+// stream: its blocks may be scheduled while that kernel finishes, and wait
+// for it in the kernel (wait_prior_grid) before reading its outputs.
+template <class Kernel, class Arg>
+cudaError_t launch_dependent(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             const Arg &arg)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, arg);
+}
+
 struct PutParams {
     __nv_bfloat16 *k_pool;
     __nv_bfloat16 *v_pool;
