@@ -110,7 +110,8 @@ typedef struct tf_streams {
     const int32_t *table;
     int32_t table_stride;
     const int32_t *lens;
-    int32_t n_streams;
+    int32_t n_streams;  /* 0: every call checks its host arguments, then does
+                         * nothing and returns TF_OK (its buffers may be null) */
     int32_t max_len;
 } tf_streams;
 
@@ -188,7 +189,8 @@ TF_API int tf_paged_attn_verify(const tf_kv_pool *pool, const tf_streams *stream
  *              above `rows` are ignored.  A row that sees no position at all
  *              (no context before the window and an empty mask) gets NaN.
  * Everything else (arguments, layouts, results, the workspace, errors) is
- * as tf_paged_attn_verify; TF_EINVAL also when tree_masks is null, and
+ * as tf_paged_attn_verify; TF_EINVAL also when tree_masks is null (with
+ * n_streams > 0), and
  * TF_EUNSUPPORTED for head dim 256 with a page_size that is not a multiple
  * of 128.  Head dim 128
  * calls with more than 64 query rows per KV head (G * rows) read each K/V

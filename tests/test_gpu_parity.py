@@ -495,3 +495,69 @@ def test_copy_state_flags_bad_pages_and_lengths():
     lens2 = torch.tensor([150, 300], dtype=torch.int32, device="cuda")   # past max_len
     tf.tf_kv_copy_state(sk, sv, st, lens2, dk, dv, st, max_len=192, status=status)
     assert int(status.item()) & tf.TF_DEV_BAD_LEN
+
+
+# --- edge cases: odd shapes, boundary lengths, empty calls, the largest chunk
+
+@pytest.mark.parametrize("d", [128, 512])
+@pytest.mark.parametrize("G,W", [(1, 1), (3, 5), (5, 3), (1, 8), (2, 7), (7, 2)])
+def test_parity_odd_group_and_rows(d, G, W):
+    """GQA ratios outside 4/8 and odd row counts: odd rows per KV head (partial
+    slots of odd size), row blocks that end mid-window."""
+    w = small_workload(d, G, 512, W, Hkv=3, seed=13000 + d + 10 * G + W)
+    run_parity(w, [1537, W, 512, 2 * W + 1], W)
+
+
+@pytest.mark.parametrize("d,G,W", [(128, 4, 1), (128, 8, 8), (512, 8, 4), (128, 4, 100)])
+def test_parity_lengths_at_the_table_bound(d, G, W):
+    """Streams exactly as long as their table can hold (len == stride * page
+    size), next to one that is a window and nothing more (len == rows)."""
+    w = small_workload(d, G, 512, W, seed=13100 + d + G + W)
+    case = synth.make_case(w, lens=[2048, W, 1024], rows=W)
+    assert case.table.shape[1] * w.page_size == 2048
+    dc = DeviceCase(case)
+    out = dc.attend()
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, W, G, w.scale, threads=8)
+    assert torch.isfinite(out).all()
+    assert max_abs(out, ref) <= TOL
+
+
+def test_calls_with_no_streams_do_nothing():
+    import verify_paged_gqa_b200 as tf
+    w = small_workload(128, 4, 512, 2, seed=13200)
+    case = synth.make_case(w, lens=[600])
+    dc = DeviceCase(case)
+    empty_t = dc.table[:0].contiguous()
+    empty_l = dc.lens[:0].contiguous()
+    q0 = dc.q[:0].contiguous()
+    out0 = torch.empty(q0.shape, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    for fn in (tf.tf_paged_attn_verify, tf.tf_paged_attn_prompt):
+        fn(dc.k_pool, dc.v_pool, empty_t, empty_l, q0, w.scale, out0, ws, 600)
+    tf.tf_paged_attn_verify_tree(dc.k_pool, dc.v_pool, empty_t, empty_l, q0,
+                                 torch.zeros((0, 2), dtype=torch.uint8, device="cuda"), w.scale,
+                                 out0, ws, 600)
+    tf.tf_kv_put_rows(dc.k_pool, dc.v_pool, empty_t, empty_l,
+                      torch.zeros((0, 2, 2, 128), dtype=torch.bfloat16, device="cuda"),
+                      torch.zeros((0, 2, 2, 128), dtype=torch.bfloat16, device="cuda"), max_len=600)
+    tf.tf_kv_copy_state(dc.k_pool, dc.v_pool, empty_t, empty_l, dc.k_pool, dc.v_pool, empty_t,
+                        max_len=600)
+    torch.cuda.synchronize()
+    assert tf.tf_workspace_status(ws) == 0
+
+
+def test_largest_prompt_chunk_sampled():
+    """A 4,096-row chunk (the largest the prompt call takes) over 4,096 + 500
+    positions, checked on sampled rows."""
+    W = 4096
+    w = small_workload(128, 4, 512, W, Hkv=2, seed=13300)
+    case = synth.make_case(w, lens=[W + 500], rows=W)
+    out = DeviceCase(case).attend().cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(13301)
+    rows = sorted(set(int(x) for x in rng.choice(W, 24, replace=False)) | {0, W - 1})
+    units = np.array([(0, r, h) for r in rows for h in (0, 5)], dtype=np.int32)
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, W, w.group, w.scale,
+                        units=units, threads=8)
+    got = np.stack([out[0, r, h] for r in rows for h in (0, 5)])
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= TOL

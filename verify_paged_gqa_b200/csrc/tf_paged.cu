@@ -183,14 +183,14 @@ int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32
     int rc = make_plan(pool, st, Hq, rows, rows_max, tree != nullptr, &plan);
     if (rc != TF_OK)
         return rc;
-    if (!q || !out || !ws || !aligned16(q) || !aligned16(out) || !aligned16(ws))
-        return TF_EINVAL;
     if (!std::isfinite(scale))
+        return TF_EINVAL;
+    if (st->n_streams == 0)
+        return TF_OK;  // nothing is read or written: the buffers may be null
+    if (!q || !out || !ws || !aligned16(q) || !aligned16(out) || !aligned16(ws))
         return TF_EINVAL;
     if (ws_bytes < plan.ws_bytes)
         return TF_ENOSPACE;
-    if (st->n_streams == 0)
-        return TF_OK;
     AttnParams &p = plan.p;
     p.k_pool = static_cast<const __nv_bfloat16 *>(pool->k_pool);
     p.v_pool = static_cast<const __nv_bfloat16 *>(pool->v_pool);
@@ -349,7 +349,7 @@ int tf_paged_attn_verify_tree(const tf_kv_pool *pool, const tf_streams *streams,
                               float scale, float *out, void *workspace, size_t workspace_bytes,
                               void *stream)
 {
-    if (!tree_masks)
+    if (streams && streams->n_streams > 0 && !tree_masks)
         return TF_EINVAL;
     return attn_call(pool, streams, q, n_q_heads, rows, 8, tree_masks, scale, out, workspace,
                      workspace_bytes, stream);
