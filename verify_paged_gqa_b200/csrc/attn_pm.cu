@@ -71,11 +71,21 @@ struct PmCfg {
     static constexpr int kFit =
         (int)((kSmemCap - 1024 - kQBytes - kPBufs * kPBytes - kSmall) / kUnit);
     static constexpr int NU = kFit > 6 ? 6 : kFit;     // ring units
+    // Head dim 128 has two MMA issuers (QK and PV, see pm_qk_issuer): one
+    // thread issues an MMA about every 130 cycles, and the 16 MMAs of a
+    // 128-position tile come close to the tile's HBM time when the power cap
+    // lowers the clock.  Its ring's slots are then split: K units in slots
+    // [0, NK), V units in [NK, NU), each part with one consumer.
+    static constexpr bool kDual = D == 128;
+    static constexpr int NK = kDual ? 2 : NU;
+    static constexpr int NV = kDual ? NU - 2 : NU;
     static_assert(kCols <= 512, "tensor memory");
-    static_assert(NU >= 2, "ring");
+    static_assert(NU >= 2 && (!kDual || NV >= 2), "ring");
     static_assert(NR == 32 || NR == 64, "row block");
     static constexpr int kSoftThreads = 4 * NR;        // 32 rows per softmax thread
-    static constexpr int kThreads = 64 + kSoftThreads; // + producer and MMA warps
+    static constexpr int kPvWarp = 2 + kSoftThreads / 32;  // the PV issuer (dual issue)
+    // + producer and MMA issuer warps
+    static constexpr int kThreads = (kDual ? 96 : 64) + kSoftThreads;
 };
 
 template <int D, int NR>
@@ -99,7 +109,8 @@ struct PmSmem {
     uint64_t s_full[2];   // S^T(t) is in tensor memory
     uint64_t p_full[2];   // the softmax warps wrote P^T(t)
     uint64_t o_done[2];   // the PV reading P^T buffer b (and every MMA before it) completed
-    uint64_t fin;
+    uint64_t fin;         // every MMA of the (QK) issuer completed
+    uint64_t fin_pv;      // every MMA of the PV issuer completed (dual issue)
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -168,10 +179,13 @@ __device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d
 {
     using C = PmCfg<D, NR>;
     constexpr uint32_t idQK = f16_idesc(128, NR, 0, 0);
+    // single issue: U counts every unit of the shared ring; dual: K units of
+    // the ring's K part (slots [0, NK))
+    constexpr int NRING = C::kDual ? C::NK : C::NU;
 #pragma unroll 1
     for (int kb = 0; kb < C::DB; ++kb) {
-        const int st = (int)(U % C::NU);
-        if (!pwait(sm, &sm.full[st], (U / C::NU) & 1u, flags, kWaitFull))
+        const int st = (int)(U % NRING);
+        if (!pwait(sm, &sm.full[st], (U / NRING) & 1u, flags, kWaitFull))
             return false;
         tc_fence_after();
         const uint32_t ka = ring0 + st * kUnit;
@@ -263,6 +277,167 @@ __device__ __forceinline__ bool pm_sees(int r, int rvis, uint32_t vis)
         return ((vis >> r) & 1u) != 0;
     else
         return r >= rvis;
+}
+
+// ---- dual issue (head dim 128) ---------------------------------------------
+
+// One lane: per segment K(0), then per tile K(t + 1) (if any) and V(t); K
+// units into the ring's K part, V units into its V part.  Page ids are read
+// two tiles ahead.
+template <int D, int NR>
+__device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> &sm)
+{
+    using C = PmCfg<D, NR>;
+    const AttnParams &p = a.p;
+    const uint64_t pol = l2_evict_first_policy();
+    uint32_t UK = 0, UV = 0;
+    bool ok = true;
+    // one unit (DB = 1) of page `page`, positions [off, off + 128), into slot st
+    auto put = [&](int st, uint32_t parity, const CUtensorMap *map, int page, int kh, int off) {
+        const bool page_ok = page >= 0 && page < p.n_pages;
+        if (!page_ok)
+            set_flag(p.flags, kDevBadPage);
+        if (!pwait(sm, &sm.empty[st], parity, p.flags, kWaitEmpty))
+            return false;
+        if (page_ok) {
+            const int y = (page * p.Hkv + kh) * p.P + off;
+            mbar_arrive_expect_tx(&sm.full[st], kUnit);
+            tma_load_2d(sm.ring[st], map, 0, y, &sm.full[st], pol);
+            tma_load_2d(sm.ring[st] + kBox, map, 64, y, &sm.full[st], pol);
+        } else {
+            mbar_arrive(&sm.full[st]);
+        }
+        return true;
+    };
+    SegCursor cur;
+    cur.init(p, sm.range);
+    WorkItem it;
+    while (ok && cur.next(p, it)) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
+        int pg0 = __ldg(trow + it.key0 / p.P);
+        int pg1 = n > 1 ? __ldg(trow + (it.key0 + PT) / p.P) : 0;
+        ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg0, it.kh, it.key0 % p.P);
+        ++UK;
+        for (int t = 0; ok && t < n; ++t) {
+            const int pos = it.key0 + t * PT;
+            const int pg2 = t + 2 < n ? __ldg(trow + (pos + 2 * PT) / p.P) : 0;
+            if (t + 1 < n) {
+                ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg1, it.kh,
+                         (pos + PT) % p.P);
+                ++UK;
+            }
+            if (ok) {
+                ok = put(C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u, &a.vmap, pg0, it.kh,
+                         pos % p.P);
+                ++UV;
+            }
+            pg0 = pg1;
+            pg1 = pg2;
+        }
+    }
+    if (!ok || sm.abort_flag) {
+        // let the copies in flight land before the CTA exits
+        for (uint32_t k = 1; k <= (UK < (uint32_t)C::NK ? UK : (uint32_t)C::NK); ++k)
+            (void)mbar_wait(&sm.full[(UK - k) % C::NK], ((UK - k) / C::NK) & 1u);
+        for (uint32_t k = 1; k <= (UV < (uint32_t)C::NV ? UV : (uint32_t)C::NV); ++k)
+            (void)mbar_wait(&sm.full[C::NK + (UV - k) % C::NV], ((UV - k) / C::NV) & 1u);
+    }
+}
+
+// One lane: S^T(T) = K Q^T into S^T buffer T % 2 once the softmax arrived on
+// p_full for tile T - 2 (it is done reading that buffer then).
+template <int D, int NR>
+__device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
+{
+    using C = PmCfg<D, NR>;
+    const AttnParams &p = a.p;
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t ring0 = smem_addr(sm.ring[0]);
+    const uint32_t q0 = smem_addr(sm.q);
+    SegCursor cur;
+    cur.init(p, sm.range);
+    WorkItem it;
+    uint32_t U = 0, T = 0, j = 0;
+    bool ok = true;
+    for (; ok && cur.next(p, it); ++j) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        ok = pwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
+        for (int t = 0; ok && t < n; ++t, ++T) {
+            if (T >= 2)
+                ok = pwait(sm, &sm.p_full[T & 1u], ((T - 2) >> 1) & 1u, p.flags, kWaitQEmpty);
+            tc_fence_after();
+            ok = ok && pm_qk(sm, U, tmem + C::kColS + (T & 1u) * NR, ring0, q0, p.flags);
+            if (!ok)
+                break;
+            umma_commit(&sm.s_full[T & 1u]);
+            if (t + 1 == n)
+                umma_commit(&sm.q_free);
+        }
+    }
+    // every MMA issued by this thread has completed once `fin` flips
+    umma_commit(&sm.fin);
+    (void)mbar_wait(&sm.fin, 0);
+}
+
+// The whole warp; lane 0 issues O^T += V^T P^T(T) once the softmax wrote
+// P^T(T).  Before the PV of a stream's last tile the warp zeroes the V rows
+// past the stream's end (their P is 0, but 0 * NaN = NaN); it is the V
+// part's only consumer, so its wait on the slot names the right phase.
+template <int D, int NR>
+__device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm, int lane)
+{
+    using C = PmCfg<D, NR>;
+    const AttnParams &p = a.p;
+    const uint32_t tmem = sm.tmem_base;
+    constexpr uint32_t idPV = f16_idesc(128, 2 * NR, 1, 1);
+    const uint32_t pt0 = smem_addr(sm.pt[0]);
+    SegCursor cur;
+    cur.init(p, sm.range);
+    WorkItem it;
+    uint32_t T = 0;
+    bool ok = true;
+    while (ok && cur.next(p, it)) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        for (int t = 0; ok && t < n; ++t, ++T) {
+            const int st = C::NK + (int)(T % C::NV);
+            if (lane == 0)
+                ok = pwait(sm, &sm.p_full[T & 1u], (T >> 1) & 1u, p.flags, kWaitQEmpty) &&
+                     pwait(sm, &sm.full[st], (T / C::NV) & 1u, p.flags, kWaitFull);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok)
+                break;
+            const int nvalid = it.len - (it.key0 + t * PT);
+            if (nvalid < PT) {
+                // every lane acquires the landed unit (its phase is complete and
+                // cannot move on before this warp releases the slot)
+                (void)mbar_wait(&sm.full[st], (T / C::NV) & 1u);
+                // rows nvalid .. 127 of both boxes: 16 chunks of 16 bytes a row
+                for (int f = lane; f < (PT - nvalid) * 16; f += 32)
+                    *reinterpret_cast<uint4 *>(sm.ring[st] + ((f >> 3) & 1) * kBox +
+                                               sw128_off(nvalid + (f >> 4), f & 7)) =
+                        make_uint4(0, 0, 0, 0);
+                fence_async_smem();
+                __syncwarp();
+            }
+            if (lane == 0) {
+                tc_fence_after();
+                const uint32_t va = smem_addr(sm.ring[st]);
+                const uint32_t pb = pt0 + (T % C::kPBufs) * C::kPBytes;
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    umma_f16(tmem + C::kColO, sw128_desc(va + s * 2048, kBox, 1024),
+                             sw128_desc(pb + s * 2048, kBox, 1024), idPV, (t > 0 || s > 0) ? 1u : 0u);
+                umma_commit(&sm.empty[st]);
+                umma_commit(&sm.o_done[T & 1u]);
+            }
+        }
+    }
+    if (lane == 0) {
+        umma_commit(&sm.fin_pv);
+        (void)mbar_wait(&sm.fin_pv, 0);
+    }
+    __syncwarp();
 }
 
 // ---- softmax warps -----------------------------------------------------------
@@ -487,7 +662,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
             }
             // --- V rows past the stream's end: zero them (0 * NaN = NaN) ----
             const int nvalid = it.len - tpos;
-            if (nvalid < PT) {
+            if (!C::kDual && nvalid < PT) {
                 // The ring slots of this tile's V units last held units of
                 // V(t - 1) or earlier (at head dim 512 the ring is shorter than
                 // a tile): wait for PV(u - 1) first, so each full-barrier wait
@@ -622,6 +797,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
             mbar_init(&sm.o_done[b], 1);
         }
         mbar_init(&sm.fin, 1);
+        mbar_init(&sm.fin_pv, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -639,13 +815,23 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     tc_fence_after();
 
     if (warp == 0) {
-        if (lane == 0)
-            ring_producer<PmCfg<D, NR>::DB, PmCfg<D, NR>::NU>(a.p, &a.kmap, &a.vmap, sm);
+        if (lane == 0) {
+            if constexpr (C::kDual)
+                pm_producer_dual<D, NR>(a, sm);
+            else
+                ring_producer<C::DB, C::NU>(a.p, &a.kmap, &a.vmap, sm);
+        }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0)
-            pm_issuer<D, NR>(a, sm);
+        if (lane == 0) {
+            if constexpr (C::kDual)
+                pm_qk_issuer<D, NR>(a, sm);
+            else
+                pm_issuer<D, NR>(a, sm);
+        }
         __syncwarp();
+    } else if (C::kDual && warp == C::kPvWarp) {
+        pm_pv_issuer<D, NR>(a, sm, lane);
     } else {
         pm_softmax<D, NR, kTree>(a, sm, warp, lane);
     }
