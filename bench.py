@@ -556,7 +556,7 @@ def run_reference(args):
     value = work / secs
     unit = oracle_unit(args.workload)
     line = {"impl": "reference", "metric": METRIC if unit == "GB/s" else PROMPT_METRIC,
-            "value": value, "unit": unit, "n_gpus": 0,
+            "value": value, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(args.workload),
