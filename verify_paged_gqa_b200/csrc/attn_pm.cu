@@ -281,9 +281,9 @@ __device__ __forceinline__ bool pm_sees(int r, int rvis, uint32_t vis)
 
 // ---- dual issue (head dim 128) ---------------------------------------------
 
-// One lane: per segment K(0), then per tile K(t + 1) (if any) and V(t); K
-// units into the ring's K part, V units into its V part.  Page ids are read
-// two tiles ahead.
+// One lane: per segment the DB units of K(0), then per tile unit kb of
+// K(t + 1) (if any) and unit kb of V(t) in turn; K units into the ring's K
+// part, V units into its V part.  Page ids are read two tiles ahead.
 template <int D, int NR>
 __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> &sm)
 {
@@ -292,8 +292,10 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
     const uint64_t pol = l2_evict_first_policy();
     uint32_t UK = 0, UV = 0;
     bool ok = true;
-    // one unit (DB = 1) of page `page`, positions [off, off + 128), into slot st
-    auto put = [&](int st, uint32_t parity, const CUtensorMap *map, int page, int kh, int off) {
+    // unit kb (dims [128 kb, 128 kb + 128)) of page `page`, positions
+    // [off, off + 128), into slot st
+    auto put = [&](int st, uint32_t parity, const CUtensorMap *map, int page, int kh, int off,
+                   int kb) {
         const bool page_ok = page >= 0 && page < p.n_pages;
         if (!page_ok)
             set_flag(p.flags, kDevBadPage);
@@ -302,8 +304,8 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
         if (page_ok) {
             const int y = (page * p.Hkv + kh) * p.P + off;
             mbar_arrive_expect_tx(&sm.full[st], kUnit);
-            tma_load_2d(sm.ring[st], map, 0, y, &sm.full[st], pol);
-            tma_load_2d(sm.ring[st] + kBox, map, 64, y, &sm.full[st], pol);
+            tma_load_2d(sm.ring[st], map, 128 * kb, y, &sm.full[st], pol);
+            tma_load_2d(sm.ring[st] + kBox, map, 128 * kb + 64, y, &sm.full[st], pol);
         } else {
             mbar_arrive(&sm.full[st]);
         }
@@ -317,20 +319,25 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
         int pg0 = __ldg(trow + it.key0 / p.P);
         int pg1 = n > 1 ? __ldg(trow + (it.key0 + PT) / p.P) : 0;
-        ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg0, it.kh, it.key0 % p.P);
-        ++UK;
+#pragma unroll 1
+        for (int kb = 0; ok && kb < C::DB; ++kb, ++UK)
+            ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg0, it.kh,
+                     it.key0 % p.P, kb);
         for (int t = 0; ok && t < n; ++t) {
             const int pos = it.key0 + t * PT;
             const int pg2 = t + 2 < n ? __ldg(trow + (pos + 2 * PT) / p.P) : 0;
-            if (t + 1 < n) {
-                ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg1, it.kh,
-                         (pos + PT) % p.P);
-                ++UK;
-            }
-            if (ok) {
-                ok = put(C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u, &a.vmap, pg0, it.kh,
-                         pos % p.P);
-                ++UV;
+#pragma unroll 1
+            for (int kb = 0; ok && kb < C::DB; ++kb) {
+                if (t + 1 < n) {
+                    ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg1, it.kh,
+                             (pos + PT) % p.P, kb);
+                    ++UK;
+                }
+                if (ok) {
+                    ok = put(C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u, &a.vmap, pg0,
+                             it.kh, pos % p.P, kb);
+                    ++UV;
+                }
             }
             pg0 = pg1;
             pg1 = pg2;
@@ -395,23 +402,28 @@ __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm,
     SegCursor cur;
     cur.init(p, sm.range);
     WorkItem it;
-    uint32_t T = 0;
+    uint32_t T = 0, UV = 0;
     bool ok = true;
     while (ok && cur.next(p, it)) {
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         for (int t = 0; ok && t < n; ++t, ++T) {
-            const int st = C::NK + (int)(T % C::NV);
             if (lane == 0)
-                ok = pwait(sm, &sm.p_full[T & 1u], (T >> 1) & 1u, p.flags, kWaitQEmpty) &&
-                     pwait(sm, &sm.full[st], (T / C::NV) & 1u, p.flags, kWaitFull);
+                ok = pwait(sm, &sm.p_full[T & 1u], (T >> 1) & 1u, p.flags, kWaitQEmpty);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            const int nvalid = it.len - (it.key0 + t * PT);
+            const uint32_t pb = pt0 + (T % C::kPBufs) * C::kPBytes;
+#pragma unroll 1
+            for (int vb = 0; ok && vb < C::DB; ++vb, ++UV) {
+            const int st = C::NK + (int)(UV % C::NV);
+            if (lane == 0)
+                ok = pwait(sm, &sm.full[st], (UV / C::NV) & 1u, p.flags, kWaitFull);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok)
                 break;
-            const int nvalid = it.len - (it.key0 + t * PT);
             if (nvalid < PT) {
                 // every lane acquires the landed unit (its phase is complete and
                 // cannot move on before this warp releases the slot)
-                (void)mbar_wait(&sm.full[st], (T / C::NV) & 1u);
+                (void)mbar_wait(&sm.full[st], (UV / C::NV) & 1u);
                 // rows nvalid .. 127 of both boxes: 16 chunks of 16 bytes a row
                 for (int f = lane; f < (PT - nvalid) * 16; f += 32)
                     *reinterpret_cast<uint4 *>(sm.ring[st] + ((f >> 3) & 1) * kBox +
@@ -423,14 +435,15 @@ __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm,
             if (lane == 0) {
                 tc_fence_after();
                 const uint32_t va = smem_addr(sm.ring[st]);
-                const uint32_t pb = pt0 + (T % C::kPBufs) * C::kPBytes;
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
-                    umma_f16(tmem + C::kColO, sw128_desc(va + s * 2048, kBox, 1024),
+                    umma_f16(tmem + C::kColO + vb * 2 * NR, sw128_desc(va + s * 2048, kBox, 1024),
                              sw128_desc(pb + s * 2048, kBox, 1024), idPV, (t > 0 || s > 0) ? 1u : 0u);
                 umma_commit(&sm.empty[st]);
-                umma_commit(&sm.o_done[T & 1u]);
             }
+            }
+            if (ok && lane == 0)
+                umma_commit(&sm.o_done[T & 1u]);
         }
     }
     if (lane == 0) {
