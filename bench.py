@@ -388,11 +388,21 @@ class Workload:
 L2_BYTES = 126 * 2**20
 
 
-def time_steps(wl, steps, warmup, barrier, sampler=None):
+def time_steps(wl, steps, warmup, barrier, sampler=None, blocks=10):
     """Device time of ``steps`` steps, and the mean per step of the attention
-    calls alone (CUDA events around each call, on the launching stream).  A
-    workload whose K/V fits in L2 gets L2 flushed (a 256 MB write) between
-    steps, outside the per-step events, and its step time is the sum of those."""
+    calls alone.
+
+    The steps run back to back with nothing between their kernels, as in a
+    serving loop (the attention kernels are programmatic dependents of the
+    kernel before them): CUDA events on the launching stream bracket runs of
+    steps, not calls.  The attention calls' own time comes from as many
+    steps that run only the attention calls (the row writes already put the
+    rows in place), also back to back; an event between a row write and the
+    call after it would keep that call from starting early.  The two kinds
+    alternate in ``blocks`` runs each, so both see the same clocks as the
+    power cap settles.  A workload whose K/V fits in L2 gets L2 flushed (a
+    256 MB write) before every step of either kind, outside that step's
+    events."""
     torch = wl.torch
     parts = wl.parts()
     flush = None
@@ -403,35 +413,44 @@ def time_steps(wl, steps, warmup, barrier, sampler=None):
     torch.cuda.synchronize()
     barrier()
     stream = torch.cuda.current_stream()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    ev = [[(mk(), mk()) for _ in parts] for _ in range(steps)]
-    sev = [(mk(), mk()) for _ in range(steps)]
+    blocks = max(1, min(blocks, steps))
+    bounds = [steps * k // blocks for k in range(blocks + 1)]
+    full = lambda: [(put(), att()) for put, att in parts]
+    attn_only = lambda: [att() for _, att in parts]
+    runs = {0: [], 1: []}   # 0: whole steps, 1: attention calls; lists of (start, end) events
+
+    def run(kind, n, i0):
+        body = full if kind == 0 else attn_only
+        if flush is None:
+            ev = (mk(), mk())
+            ev[0].record(stream)
+            for _ in range(n):
+                body()
+            ev[1].record(stream)
+            runs[kind].append(ev)
+        else:
+            for i in range(i0, i0 + n):
+                flush.fill_(i & 255)
+                ev = (mk(), mk())
+                ev[0].record(stream)
+                body()
+                ev[1].record(stream)
+                runs[kind].append(ev)
+
     if sampler:
         sampler.mark()
-    start.record(stream)
-    for i in range(steps):
-        if flush is not None:
-            flush.fill_(i & 255)
-        sev[i][0].record(stream)
-        for (put, att), (a, b) in zip(parts, ev[i]):
-            put()
-            a.record(stream)
-            att()
-            b.record(stream)
-        sev[i][1].record(stream)
-    end.record(stream)
+    for k in range(blocks):
+        n = bounds[k + 1] - bounds[k]
+        run(0, n, bounds[k])
+        run(1, n, bounds[k])
     torch.cuda.synchronize()
     if sampler:
         sampler.mark()
     barrier()
-    if flush is not None:
-        total_ms = sum(a.elapsed_time(b) for a, b in sev)
-    else:
-        total_ms = start.elapsed_time(end)
-    attn_ms = [sum(a.elapsed_time(b) for a, b in step) for step in ev]
-    return total_ms, statistics.mean(attn_ms)
+    total_ms = sum(a.elapsed_time(b) for a, b in runs[0])
+    attn_ms = sum(a.elapsed_time(b) for a, b in runs[1]) / steps
+    return total_ms, attn_ms
 
 
 def time_e2e(wl, steps, warmup, barrier):

@@ -68,11 +68,14 @@ size_t ws_part_offset(int S)
 
 // Entry tiles per unit (plan.cuh), measured: at head dim 512 a unit start
 // costs about 8 tiles' worth of streaming (the ring holds less than one
-// tile, so the pipeline drains and refills); the CUDA-core decode kernel's
-// segment starts overlap with its deep ring and cost nothing measurable.
+// tile, so the pipeline drains and refills); the prompt kernel's split
+// units (more than 64 rows per KV head over long contexts) pay its serial
+// epilogue and its query load, about 8 of its tiles; the CUDA-core decode
+// kernel's segment starts overlap with its deep ring and cost nothing
+// measurable.
 constexpr int kEntryPm512 = 8;
 constexpr int kEntryPm128 = 6;
-constexpr int kEntryPrompt = 4;
+constexpr int kEntryPrompt = 8;
 constexpr int kEntrySimt = 0;
 
 struct Plan {
