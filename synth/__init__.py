@@ -154,6 +154,8 @@ WORKLOADS = {
     # smaller copies of the decode and verify workloads for profiler captures
     # (still larger than the 126 MB L2)
     "decode_12x8k": Workload("decode_12x8k", 12, 8, 4, 128, 512, 1, seed=6, lens=(8192,) * 12),
+    "decode_12x8k_p37": Workload("decode_12x8k_p37", 12, 8, 4, 128, 37, 1, seed=13,
+                                 lens=(8192,) * 12),
     "verify_4x16k": Workload("verify_4x16k", 4, 4, 8, 128, 512, 8, seed=7, lens=(16384,) * 4),
 }
 

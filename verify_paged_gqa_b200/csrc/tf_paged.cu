@@ -118,10 +118,15 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     p.W = rows;
     p.M = static_cast<int32_t>(M);
     p.has_tree = tree ? 1 : 0;
-    // More than one CUDA-core row block of rows sharing a KV head: a dense
-    // QK^T / PV tile for the tensor cores.  Up to 64 rows (128 at head dim
-    // 512 in blocks of 32) go with the positions on the MMA's M; larger
-    // blocks with the rows there.
+    // Rows sharing a KV head go to the tensor cores as a dense QK^T / PV
+    // tile: up to 64 rows (any count at head dims 256 and 512, in blocks of
+    // 32) with the positions on the MMA's M, larger blocks with the rows
+    // there.  At head dim 128 that holds for a single CUDA-core row block
+    // too (decode at GQA 4): its two MMA issuers keep pace with HBM at any
+    // clock, where the CUDA-core kernel's FMAs fall behind under the power
+    // cap (12 x 40,960 decode: 341 -> 296 us per call).  Head dim 512 keeps
+    // such calls on the CUDA-core kernel, and so do pages whose size is not
+    // a multiple of 128.
     plan->kernel = Kernel::kSimt;
     p.RB = kSimtRows;
     if (tree) {
@@ -141,7 +146,7 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
             return TF_EUNSUPPORTED;
         plan->kernel = Kernel::kPm;
         p.RB = nr;
-    } else if (M > kSimtRows) {
+    } else if (M > kSimtRows || p.D == 128) {
         const int nr = pm_rows(p);
         if (nr > 0) {
             plan->kernel = Kernel::kPm;
