@@ -1,7 +1,9 @@
 // attn_pm.cu -- split-context paged attention on the 5th-generation tensor
 // cores with the key positions on the MMA's M dimension ("position-major"),
 // for row blocks of up to 64 query rows: draft-verify windows, decode at
-// GQA 8, and every head dim 256 or 512 call.
+// head dim 128 (a GQA 4 decode block pads to 32 rows: an MMA instruction
+// costs the same for any N up to 128), every head dim 256 call, and head
+// dim 512 calls with more than four rows per KV head.
 //
 // TensorFold #1620 ("Kolibri-1's full layers take their K/V from pages of
 // the core pool"), opening comment, "Reads": decode, verify and prompt rows

@@ -1,6 +1,7 @@
 // attn_simt.cu -- split-context paged attention on CUDA cores, for row
-// blocks of four query rows (single-row decode at GQA 4, and any small
-// row count).
+// blocks of four query rows: head dim 512 calls with up to four rows per KV
+// head (decode at GQA <= 4), and every call whose page size is not a
+// multiple of 128 (the tensor-core kernels' tiles stay inside a page).
 //
 // TensorFold #1620 ("Kolibri-1's full layers take their K/V from pages of
 // the core pool"): decode reads keys through the page table, split across
