@@ -79,7 +79,7 @@ extern "C" {
 /* Status codes returned by every call. */
 #define TF_OK 0
 #define TF_EINVAL 1        /* a NULL pointer, a bad size or an inconsistent shape */
-#define TF_EUNSUPPORTED 2  /* a shape this build has no kernel for (head_dim, page_size) */
+#define TF_EUNSUPPORTED 2  /* a shape this library has no kernel for (head_dim, page_size) */
 #define TF_ENOSPACE 3      /* the workspace is smaller than tf_paged_attn_workspace_bytes */
 #define TF_ECUDA 4         /* a CUDA launch or query failed */
 

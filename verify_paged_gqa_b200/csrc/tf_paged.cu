@@ -395,7 +395,7 @@ const char *tf_status_str(int status)
     case TF_EINVAL:
         return "TF_EINVAL: invalid argument";
     case TF_EUNSUPPORTED:
-        return "TF_EUNSUPPORTED: shape not supported by this build";
+        return "TF_EUNSUPPORTED: shape not supported by this library";
     case TF_ENOSPACE:
         return "TF_ENOSPACE: workspace too small";
     case TF_ECUDA:
