@@ -109,6 +109,10 @@ def throughput(wl, ms, world=1):
     return world * wl.bytes_per_step / (ms * 1e-3) / 1e9, "GB/s"
 
 
+NOMINAL_HBM_GBS = 8000.0        # B200 HBM3e, vendor figure (DGX)
+NOMINAL_TENSOR_TFLOPS = 2250.0  # B200 dense bf16, vendor figure
+
+
 def roofline(wl, attn_ms):
     """The attention calls (partial + merge kernels) of one step against the bound
     that limits them."""
@@ -119,9 +123,11 @@ def roofline(wl, attn_ms):
     else:
         peak, src = hbm_peak()
         bound = "hbm"
+    nominal = NOMINAL_TENSOR_TFLOPS if wl.w.prompt_len else NOMINAL_HBM_GBS
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak, "traffic": recorded_traffic(wl.name),
-            "kernel": "attention calls (partial + merge)", "peak_source": src}
+            "kernel": "attention calls (partial + merge)", "peak_source": src,
+            "peak_nominal": nominal, "frac_nominal": achieved / nominal}
 
 
 def measure_other(name, args, barrier, dist, world, local):
@@ -185,10 +191,19 @@ def measure_state_copy(args, barrier, dist, world, local, name="decode_12x40k"):
         ms = t.item()
     if int(status.item()) != 0:
         raise RuntimeError(f"state copy status {int(status.item()):#x}")
-    # every copied byte checked once, after timing: the destination holds the source's rows
-    n_full = int(wl.lens_np[0]) // w.page_size      # stream 0's full pages
-    ok = all(torch.equal(dk[t2[0, i]], wl.k_pool[wl.table[0, i]])
-             for i in sorted({0, n_full // 2, n_full - 1}) if n_full > 0)
+    # after timing, a sample: K and V of the first, middle and last page of the
+    # first and the last stream (the used slots of a partial last page only)
+    # hold the source's bytes
+    P = w.page_size
+    ok = True
+    for s in sorted({0, len(wl.lens_np) - 1}):
+        n = int(wl.lens_np[s])
+        n_pages_s = (n + P - 1) // P
+        for i in sorted({0, n_pages_s // 2, n_pages_s - 1}):
+            used = min(P, n - i * P)
+            src_pg, dst_pg = int(wl.table[s, i]), int(t2[s, i])
+            ok = ok and torch.equal(dk[dst_pg, :, :used], wl.k_pool[src_pg, :, :used])
+            ok = ok and torch.equal(dv[dst_pg, :, :used], wl.v_pool[src_pg, :, :used])
     moved = 2 * kv_bytes(wl.lens_np, w.n_kv_heads, w.head_dim)      # read + write
     gbs = world * moved / (ms * 1e-3) / 1e9
     peak, src = hbm_peak()
@@ -197,7 +212,7 @@ def measure_state_copy(args, barrier, dist, world, local, name="decode_12x40k"):
            "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peak, "unit": "GB/s",
                         "frac": gbs / world / peak, "traffic": None, "kernel": "kv_copy_kernel",
                         "peak_source": src},
-           "check": "sampled pages equal" if ok else "MISMATCH",
+           "check": "K and V of 3 pages of the first and last stream equal" if ok else "MISMATCH",
            "gpu_launches": args.steps,
            "config": {"workload": label, "streams": len(wl.lens_np), "context": int(wl.lens_np.max()),
                       "kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "page_size": w.page_size,
@@ -604,6 +619,36 @@ def workload_config(name):
     return cfg
 
 
+def summary(line):
+    """The headline figures of every workload the run measured, compact, so that
+    they close the JSON line: per workload its value per step, the attention
+    calls' fraction of the measured peak ("frac") and of the vendor's nominal
+    peak ("frac_nominal"), and verify tokens/s where the workload has windows."""
+    def one(d):
+        r = d["roofline"]
+        s = {"value": round(d["value"], 1), "unit": d["unit"],
+             "ms_per_step": round(d["ms_per_step"], 4), "attn_ms": round(d.get("attn_ms", 0.0), 4),
+             "attn_achieved": round(r["achieved"], 1), "frac": round(r["frac"], 3),
+             "frac_nominal": round(r["frac_nominal"], 3)}
+        if "verify_tokens_per_s" in d:
+            s["verify_tokens_per_s"] = round(d["verify_tokens_per_s"])
+        return s
+    out = {line["config"]["workload"]: one(line)}
+    for key in ("verify", "hd512", "prompt"):
+        if key in line:
+            out[line[key]["workload"]] = one(line[key])
+    for v in line.get("variants", []):
+        out[v["workload"]] = {"value": round(v["value"], 1), "frac": round(v["roofline"]["frac"], 3),
+                              "frac_nominal": round(v["roofline"]["frac_nominal"], 3)}
+    if "state_copy" in line:
+        out[line["state_copy"]["workload"]] = {"value": round(line["state_copy"]["value"], 1),
+                                               "frac": round(line["state_copy"]["roofline"]["frac"], 3),
+                                               "check": "MISMATCH" if line["state_copy"]["check"] == "MISMATCH" else "ok"}
+    out["peaks"] = {"hbm_gbs": hbm_peak()[0], "bf16_tflops_sustained": tensor_peak()[0],
+                    "hbm_nominal_gbs": NOMINAL_HBM_GBS, "bf16_nominal_tflops": NOMINAL_TENSOR_TFLOPS}
+    return out
+
+
 # --------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
@@ -706,6 +751,8 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+    # last key of the line: the headline figures of every workload measured
+    line["summary"] = summary(line)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0

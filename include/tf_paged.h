@@ -149,7 +149,13 @@ TF_API int tf_kv_copy_state(const tf_kv_pool *src_pool, const tf_streams *src,
                             int32_t dst_table_stride, uint32_t *status, void *stream);
 
 /* Workspace bytes an attention call with these arguments needs on the
- * current device (0 on a bad argument), for any of the attention calls
+ * current device (0 on a bad argument).  Follows the scratch convention of
+ * the metrale page "metrale_model_arch/glm5next_dsa/select.rs": scratch is
+ * owned by the caller, sized once from the largest shape it will run and
+ * reused across steps (the DsaSelectScratch doc comment), and a call whose
+ * plan needs more than was given fails before any launch instead of
+ * overrunning it (DsaSelectScratch::fits; here TF_ENOSPACE).  The figure is
+ * for any of the attention calls
  * with these arguments (tf_paged_attn_verify_tree included).  The workspace holds split-context
  * partial results and, in its first 4 bytes, the device status word, which
  * the calls only OR bits into: zero those 4 bytes once after allocating
@@ -233,10 +239,16 @@ TF_API int tf_paged_attn_decode_noalloc(const tf_kv_pool *pool,
 
 /* Reads the workspace's device status word (TF_DEV_* bits accumulated by
  * the attention calls since the last read) into *flags and clears it.
- * Synchronises `stream`.  Returns TF_OK, TF_EINVAL or TF_ECUDA. */
+ * Synchronises `stream`.  Returns TF_OK, TF_EINVAL or TF_ECUDA.
+ * The source pages have no counterpart of this call: their launchers check
+ * host arguments only (the select.rs page's plan and fits), while lens and
+ * table here are device data that only the kernels can check. */
 TF_API int tf_workspace_status(void *workspace, uint32_t *flags, void *stream);
 
-/* A static, human-readable name for a status code. */
+/* A static, human-readable name for a status code.  The select.rs page's
+ * plan and fits refuse a bad shape or a short scratch with a message that
+ * names what was wrong; a C caller gets the code from the call and its name
+ * from here. */
 TF_API const char *tf_status_str(int status);
 
 #ifdef __cplusplus

@@ -15,17 +15,26 @@ def bf16_tensor(u16, device="cuda"):
     return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
 
 
-def nan_pool(n_pages, w):
+def nan_pool(n_pages, w, fill="nan"):
+    """K and V pools whose every slot holds NaN (``fill="nan"``), zero or
+    random bits (``"random"``: NaN and infinity patterns included), before the
+    streams' rows are written."""
     shape = (n_pages, w.n_kv_heads, w.page_size, w.head_dim)
-    return (torch.full(shape, float("nan"), dtype=torch.bfloat16, device="cuda"),
-            torch.full(shape, float("nan"), dtype=torch.bfloat16, device="cuda"))
+    if fill == "random":
+        g = torch.Generator(device="cuda")
+        g.manual_seed(n_pages * 1000 + w.head_dim)
+        return tuple(torch.randint(-2**15, 2**15, shape, dtype=torch.int16, device="cuda",
+                                   generator=g).view(torch.bfloat16) for _ in range(2))
+    value = float("nan") if fill == "nan" else 0.0
+    return (torch.full(shape, value, dtype=torch.bfloat16, device="cuda"),
+            torch.full(shape, value, dtype=torch.bfloat16, device="cuda"))
 
 
 class DeviceCase:
     """Pools, table and lens on the GPU for one synth.Case.  Every stream's rows
     are written with tf_kv_put_rows (one call per stream, all its positions)."""
 
-    def __init__(self, case: synth.Case, table=None, n_pages=None):
+    def __init__(self, case: synth.Case, table=None, n_pages=None, fill="nan"):
         import verify_paged_gqa_b200 as tf
         self.tf = tf
         self.case = case
@@ -33,7 +42,7 @@ class DeviceCase:
         self.w = w
         table = case.table if table is None else table
         n_pages = case.n_pages if n_pages is None else n_pages
-        self.k_pool, self.v_pool = nan_pool(n_pages, w)
+        self.k_pool, self.v_pool = nan_pool(n_pages, w, fill)
         self.table = torch.from_numpy(np.ascontiguousarray(table, dtype=np.int32)).cuda()
         self.lens = torch.from_numpy(np.ascontiguousarray(case.lens, dtype=np.int32)).cuda()
         self.max_len = int(case.lens.max())

@@ -867,21 +867,11 @@ cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
     a.p = p;
     if (!make_pool_map(&a.kmap, p.k_pool, p, PT) || !make_pool_map(&a.vmap, p.v_pool, p, PT))
         return cudaErrorInvalidValue;
-    static bool configured[kMaxDevices] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<bool> configured[kMaxDevices];
+    constexpr size_t bytes = pm_smem_bytes<D, NR>();
+    const cudaError_t e = set_smem_limit_once(attn_pm_kernel<D, NR, kTree>, bytes, configured);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
-    constexpr size_t bytes = pm_smem_bytes<D, NR>();
-    if (!configured[dev]) {
-        e = cudaFuncSetAttribute(attn_pm_kernel<D, NR, kTree>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)bytes);
-        if (e != cudaSuccess)
-            return e;
-        configured[dev] = true;
-    }
     return launch_dependent(attn_pm_kernel<D, NR, kTree>, dim3(grid), dim3(PmCfg<D, NR>::kThreads),
                             bytes, stream, a);
 }

@@ -492,20 +492,10 @@ cudaError_t launch_attn_prompt(const AttnParams &p, int grid, cudaStream_t strea
     a.p = p;
     if (!make_pool_map(&a.kmap, p.k_pool, p, PT) || !make_pool_map(&a.vmap, p.v_pool, p, PT))
         return cudaErrorInvalidValue;
-    static bool configured[kMaxDevices] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<bool> configured[kMaxDevices];
+    const cudaError_t e = set_smem_limit_once(attn_prompt_kernel, kPrSmemBytes, configured);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
-    if (!configured[dev]) {
-        e = cudaFuncSetAttribute(attn_prompt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kPrSmemBytes);
-        if (e != cudaSuccess)
-            return e;
-        configured[dev] = true;
-    }
     return launch_dependent(attn_prompt_kernel, dim3(grid), dim3(kThreads), kPrSmemBytes, stream, a);
 }
 

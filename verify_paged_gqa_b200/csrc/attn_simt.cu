@@ -715,20 +715,10 @@ template <int D, bool kTree>
 cudaError_t launch_simt(const AttnParams &p, int grid, cudaStream_t stream)
 {
     const size_t smem = simt_smem_bytes<D>();
-    static bool configured[kMaxDevices] = {};  // the attribute is set once per device
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::atomic<bool> configured[kMaxDevices];
+    const cudaError_t e = set_smem_limit_once(attn_simt_kernel<D, kTree>, smem, configured);
     if (e != cudaSuccess)
         return e;
-    if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
-    if (!configured[dev]) {
-        e = cudaFuncSetAttribute(attn_simt_kernel<D, kTree>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        if (e != cudaSuccess)
-            return e;
-        configured[dev] = true;
-    }
     return launch_dependent(attn_simt_kernel<D, kTree>, dim3(grid), dim3(simt_threads<D>()), smem,
                             stream, p);
 }

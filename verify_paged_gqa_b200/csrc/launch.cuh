@@ -3,7 +3,30 @@
 
 #include "common.cuh"
 
+#include <atomic>
+
 namespace tfp {
+
+// Raises `kernel`'s dynamic shared memory limit to `bytes`, once per device
+// (done[dev] records it).  Host threads making their first launches at once
+// may each set the same attribute, which is harmless; the flags are atomics,
+// so that race is well defined.
+template <class Kernel>
+cudaError_t set_smem_limit_once(Kernel kernel, size_t bytes, std::atomic<bool> (&done)[kMaxDevices])
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    if (done[dev].load(std::memory_order_acquire))
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess)
+        done[dev].store(true, std::memory_order_release);
+    return e;
+}
 
 // Launches `kernel` as a programmatic dependent of the previous kernel in the
 // stream: its blocks may be scheduled while that kernel finishes, and wait

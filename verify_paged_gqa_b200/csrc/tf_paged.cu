@@ -8,26 +8,30 @@
 #include "launch.cuh"
 #include "plan.cuh"
 
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
 namespace tfp {
 namespace {
 
+// The SM count of the current device, queried once per device.  Host threads
+// making their first calls at once may each query it and store the same
+// value; the atomics keep that race well defined.
 int device_sm_count(int *sms)
 {
-    static int cached[kMaxDevices] = {};
+    static std::atomic<int> cached[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return TF_ECUDA;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             n <= 0)
             return TF_ECUDA;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    *sms = cached[dev];
+    *sms = n;
     return TF_OK;
 }
 
@@ -457,7 +461,13 @@ extern "C" int tf_paged_attn_decode_noalloc(const tf_kv_pool *pool, const tf_str
     int rc = make_plan(pool, streams, n_q_heads, 1, 1, false, &plan);
     if (rc != TF_OK)
         return rc;
-    if (!q || !out || !aligned16(q) || !aligned16(out) || !std::isfinite(scale))
+    if (!std::isfinite(scale))
+        return TF_EINVAL;
+    // as tf_paged_attn_decode: a call with no streams reads and writes
+    // nothing, and its buffers may be null
+    if (streams->n_streams == 0)
+        return TF_OK;
+    if (!q || !out || !aligned16(q) || !aligned16(out))
         return TF_EINVAL;
     if (plan.ws_bytes > kStaticScratchBytes)
         return TF_ENOSPACE;
@@ -465,14 +475,11 @@ extern "C" int tf_paged_attn_decode_noalloc(const tf_kv_pool *pool, const tf_str
     rc = static_scratch_address(&ws);
     if (rc != TF_OK)
         return rc;
-    if (streams->n_streams == 0)
-        return TF_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // The status word is the only part of the scratch that must start at
-    // zero (the kernels OR bits into it); the partials are written before
-    // they are read.
-    if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess)
-        return TF_ECUDA;
+    // Nothing in the scratch needs clearing: the kernels write every partial
+    // and the header's tile counts before reading them.  The header's status
+    // and wait-site words only collect bits (ORed in by the kernels) that no
+    // kernel reads and this call does not report, so they are left as they
+    // are; their contents are unspecified.
     return attn_call(pool, streams, q, n_q_heads, 1, 1, nullptr, scale, out, ws, kStaticScratchBytes,
                      stream);
 }
