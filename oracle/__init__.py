@@ -41,12 +41,19 @@ _lock = threading.Lock()
 _lib = None
 
 
-def compile_source(src: str, out: str) -> str:
-    """Compile one C source of the oracle into a shared library (gcc, -O2, no fast-math)."""
+SANITIZE_FLAGS = ["-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
+                  "-fno-omit-frame-pointer", "-g"]
+
+
+def compile_source(src: str, out: str, sanitize: bool = False) -> str:
+    """Compile one C source of the oracle into a shared library (gcc, -O2, no
+    fast-math); ``sanitize`` adds AddressSanitizer and UndefinedBehaviorSanitizer
+    (the process that loads it must preload libasan)."""
     tmp = out + f".tmp{os.getpid()}"
     subprocess.check_call(
         ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-Wall", "-Wextra",
-         "-fno-fast-math", "-ffp-contract=off", src, "-o", tmp, "-lm", "-lpthread"])
+         "-fno-fast-math", "-ffp-contract=off", *(SANITIZE_FLAGS if sanitize else []),
+         src, "-o", tmp, "-lm", "-lpthread"])
     os.replace(tmp, out)
     return out
 
@@ -78,10 +85,12 @@ def open_library(path: str):
 
 
 def _load():
+    """The oracle library: TF_ORACLE_LIB names another build of tf_oracle.c (a
+    sanitizer build, for instance), else the default one is built and used."""
     global _lib
     with _lock:
         if _lib is None:
-            _lib = open_library(build())
+            _lib = open_library(os.environ.get("TF_ORACLE_LIB") or build())
     return _lib
 
 

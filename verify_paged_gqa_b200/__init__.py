@@ -12,7 +12,7 @@ _EXPORTS = (
     "TF_ECUDA", "TF_EUNSUPPORTED", "TF_OK", "TFError", "library_path", "raw",
     "tf_kv_copy_state", "tf_kv_put_rows", "tf_paged_attn_decode", "tf_paged_attn_prompt", "tf_paged_attn_verify",
     "tf_paged_attn_verify_tree", "tf_paged_attn_workspace_bytes", "tf_status_str",
-    "tf_workspace_status",
+    "tf_workspace_status", "tf_testing_paged_attn",
 )
 __all__ = list(_EXPORTS)
 

@@ -25,7 +25,9 @@ import re
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libtfpaged.so")
+# TFPAGED_LIBRARY names another build of the library (a sanitizer build, for
+# instance); by default the one built in place is loaded.
+library_path = os.environ.get("TFPAGED_LIBRARY") or os.path.join(_HERE, "libtfpaged.so")
 
 
 def _header_value(name: str) -> int:
@@ -85,6 +87,9 @@ raw.tf_paged_attn_verify_tree.restype = ctypes.c_int
 raw.tf_kv_copy_state.argtypes = [_P(tf_kv_pool), _P(tf_streams), _P(tf_kv_pool), _vp, _i32, _vp,
                                  _vp]
 raw.tf_kv_copy_state.restype = ctypes.c_int
+raw.tf_testing_paged_attn.argtypes = [_P(tf_kv_pool), _P(tf_streams), _vp, _i32, _i32, _f32,
+                                      _vp, _vp, _sz, ctypes.c_int64, _i32, _vp]
+raw.tf_testing_paged_attn.restype = ctypes.c_int
 raw.tf_workspace_status.argtypes = [_vp, _P(ctypes.c_uint32), _vp]
 raw.tf_workspace_status.restype = ctypes.c_int
 raw.tf_status_str.argtypes = [ctypes.c_int]
@@ -231,6 +236,25 @@ def tf_paged_attn_prompt(k_pool, v_pool, table, lens, q, scale, out, workspace, 
     """A causal chunk of q.shape[1] prompt rows per stream (the last rows of each stream)."""
     return _attn(raw.tf_paged_attn_prompt, "tf_paged_attn_prompt", k_pool, v_pool, table, lens,
                  q, scale, out, workspace, max_len, stream, with_rows=True)
+
+
+def tf_testing_paged_attn(k_pool, v_pool, table, lens, q, scale, out, workspace, max_len,
+                          wait_limit_cycles, withhold, stream=None):
+    """The test hook of include/tf_paged_testing.h: a causal attention call of
+    q.shape[1] rows per stream with a shorter wait limit and, with
+    ``withhold=1``, one arrival withheld in CTA 0 so that a wait runs out."""
+    _need(q, torch.bfloat16, 4, "q")
+    _need(out, torch.float32, 4, "out")
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have q's shape")
+    pool, st = _pool(k_pool, v_pool), _streams(table, lens, max_len)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(raw.tf_testing_paged_attn(ctypes.byref(pool), ctypes.byref(st), q.data_ptr(),
+                                     q.shape[2], q.shape[1], float(scale), out.data_ptr(),
+                                     workspace.data_ptr(), ws_bytes, int(wait_limit_cycles),
+                                     int(withhold), _stream(stream)),
+           "tf_testing_paged_attn")
+    return out
 
 
 def tf_workspace_status(workspace, stream=None) -> int:

@@ -46,15 +46,29 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and not verbose and up_to_date():
+# host-compiler flags of the sanitizer build (one per -Xcompiler: nvcc splits
+# an -Xcompiler value at commas)
+SANITIZE = ["-fsanitize=address", "-fsanitize=undefined", "-fno-sanitize-recover=undefined",
+            "-fno-omit-frame-pointer"]
+
+
+def build(verbose: bool = False, force: bool = False, sanitize: bool = False) -> str:
+    """Compile and link the library; returns its path.  ``sanitize`` builds a
+    separate copy (_build/asan/libtfpaged_asan.so) whose host code carries
+    AddressSanitizer and UndefinedBehaviorSanitizer (device code is
+    unchanged; the process that loads it must preload libasan)."""
+    if not sanitize and not force and not verbose and up_to_date():
         return LIB
-    os.makedirs(BUILD, exist_ok=True)
+    build_dir = os.path.join(ROOT, "_build", "asan") if sanitize else BUILD
+    lib = os.path.join(build_dir, "libtfpaged_asan.so") if sanitize else LIB
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if verbose else []
+    if sanitize:
+        extra += [f"-Xcompiler={f}" for f in SANITIZE] + ["-g"]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+        obj = os.path.join(build_dir, src.replace(".cu", ".o"))
         cmd = [cc, *ARCH, *FLAGS, *extra, "-c", os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -64,17 +78,18 @@ def build(verbose: bool = False, force: bool = False) -> str:
     with concurrent.futures.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         results = list(ex.map(compile_one, SOURCES))
     log = "".join(out for _, out in results)
-    with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+    with open(os.path.join(build_dir, "ptxas.log"), "w") as f:
         f.write(log)
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [cc, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results], "-lcudart"]
+    tmp = lib + f".tmp{os.getpid()}"
+    link_extra = ["-Xcompiler=-fsanitize=address", "-Xcompiler=-fsanitize=undefined"] if sanitize else []
+    cmd = [cc, *ARCH, "-shared", *link_extra, "-o", tmp, *[o for o, _ in results], "-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     if verbose:
         sys.stdout.write(log)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":

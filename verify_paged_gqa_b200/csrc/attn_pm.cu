@@ -115,6 +115,7 @@ struct PmSmem {
     uint64_t fin_pv;      // every MMA of the PV issuer completed (dual issue)
     uint32_t tmem_base;
     volatile int abort_flag;
+    long long wait_limit;  // cycles a pipeline wait may take (the call's)
 };
 
 template <int D, int NR>
@@ -268,7 +269,7 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
     }
     // every MMA issued by this thread has completed once `fin` flips
     umma_commit(&sm.fin);
-    (void)mbar_wait(&sm.fin, 0);
+    (void)mbar_wait(&sm.fin, 0, sm.wait_limit);
 }
 
 // Whether the thread's row R0 + r sees its position (see the tile loop).
@@ -321,10 +322,13 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
         int pg0 = __ldg(trow + it.key0 / p.P);
         int pg1 = n > 1 ? __ldg(trow + (it.key0 + PT) / p.P) : 0;
+        // (UK and UV count the units actually issued)
 #pragma unroll 1
-        for (int kb = 0; ok && kb < C::DB; ++kb, ++UK)
+        for (int kb = 0; ok && kb < C::DB; ++kb) {
             ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg0, it.kh,
                      it.key0 % p.P, kb);
+            UK += ok ? 1u : 0u;
+        }
         for (int t = 0; ok && t < n; ++t) {
             const int pos = it.key0 + t * PT;
             const int pg2 = t + 2 < n ? __ldg(trow + (pos + 2 * PT) / p.P) : 0;
@@ -333,24 +337,27 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
                 if (t + 1 < n) {
                     ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg1, it.kh,
                              (pos + PT) % p.P, kb);
-                    ++UK;
+                    UK += ok ? 1u : 0u;
                 }
                 if (ok) {
                     ok = put(C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u, &a.vmap, pg0,
                              it.kh, pos % p.P, kb);
-                    ++UV;
+                    UV += ok ? 1u : 0u;
                 }
             }
             pg0 = pg1;
             pg1 = pg2;
         }
     }
-    if (!ok || sm.abort_flag) {
-        // let the copies in flight land before the CTA exits
+    {
+        // Let the copies in flight land before the CTA can exit.  On the
+        // normal path every unit was consumed and these phases are complete;
+        // after another role gave up, some may still be in flight.
         for (uint32_t k = 1; k <= (UK < (uint32_t)C::NK ? UK : (uint32_t)C::NK); ++k)
-            (void)mbar_wait(&sm.full[(UK - k) % C::NK], ((UK - k) / C::NK) & 1u);
+            (void)mbar_wait(&sm.full[(UK - k) % C::NK], ((UK - k) / C::NK) & 1u, sm.wait_limit);
         for (uint32_t k = 1; k <= (UV < (uint32_t)C::NV ? UV : (uint32_t)C::NV); ++k)
-            (void)mbar_wait(&sm.full[C::NK + (UV - k) % C::NV], ((UV - k) / C::NV) & 1u);
+            (void)mbar_wait(&sm.full[C::NK + (UV - k) % C::NV], ((UV - k) / C::NV) & 1u,
+                            sm.wait_limit);
     }
 }
 
@@ -386,7 +393,7 @@ __device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
     }
     // every MMA issued by this thread has completed once `fin` flips
     umma_commit(&sm.fin);
-    (void)mbar_wait(&sm.fin, 0);
+    (void)mbar_wait(&sm.fin, 0, sm.wait_limit);
 }
 
 // The whole warp; lane 0 issues O^T += V^T P^T(T) once the softmax wrote
@@ -425,7 +432,7 @@ __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm,
             if (nvalid < PT) {
                 // every lane acquires the landed unit (its phase is complete and
                 // cannot move on before this warp releases the slot)
-                (void)mbar_wait(&sm.full[st], (UV / C::NV) & 1u);
+                (void)mbar_wait(&sm.full[st], (UV / C::NV) & 1u, sm.wait_limit);
                 // rows nvalid .. 127 of both boxes: 16 chunks of 16 bytes a row
                 for (int f = lane; f < (PT - nvalid) * 16; f += 32)
                     *reinterpret_cast<uint4 *>(sm.ring[st] + ((f >> 3) & 1) * kBox +
@@ -450,7 +457,7 @@ __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm,
     }
     if (lane == 0) {
         umma_commit(&sm.fin_pv);
-        (void)mbar_wait(&sm.fin_pv, 0);
+        (void)mbar_wait(&sm.fin_pv, 0, sm.wait_limit);
     }
     __syncwarp();
 }
@@ -737,7 +744,8 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
+            // (the test switch: every CTA withholds its first tile's arrival)
+            if (lane == 0 && !(p.withhold && u == 0))
                 mbar_arrive(&sm.p_full[u & 1u]);
         }
 
@@ -814,6 +822,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
         mbar_init(&sm.fin, 1);
         mbar_init(&sm.fin_pv, 1);
         sm.abort_flag = 0;
+        sm.wait_limit = a.p.wait_limit;
         fence_mbar_init();
     }
     if (warp == 1) {

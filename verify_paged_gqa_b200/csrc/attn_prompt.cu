@@ -74,6 +74,7 @@ struct PrSmem {
     CtaRange range;
     uint32_t tmem_base;
     volatile int abort_flag;
+    long long wait_limit;  // cycles a pipeline wait may take (the call's)
 };
 
 constexpr size_t kPrSmemBytes = sizeof(PrSmem) + 1024;  // + alignment slack
@@ -170,7 +171,7 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
     }
     // every MMA issued by this thread has completed once `fin` flips
     umma_commit(&sm.fin);
-    (void)mbar_wait(&sm.fin, 0);
+    (void)mbar_wait(&sm.fin, 0, sm.wait_limit);
 }
 
 // ---- softmax warps -----------------------------------------------------------
@@ -372,7 +373,8 @@ __device__ __forceinline__ void pr_softmax(const PrArgs &a, PrSmem &sm, int warp
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
+            // (the test switch: every CTA withholds its first tile's arrival)
+            if (lane == 0 && !(p.withhold && u == 0))
                 mbar_arrive(&sm.p_full);
         }
 
@@ -439,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.fin, 1);
         sm.abort_flag = 0;
+        sm.wait_limit = a.p.wait_limit;
         fence_mbar_init();
     }
     if (warp == 1) {

@@ -102,6 +102,7 @@ struct SimtSmem {
     int w_count;           // warps parked for the current segment
     CtaRange range;        // this CTA's tiles
     volatile int abort_flag;
+    long long wait_limit;  // cycles a pipeline wait may take (the call's)
 };
 
 template <int D>
@@ -149,7 +150,7 @@ __device__ __forceinline__ bool wait_or_abort(SimtSmem<D> &sm, uint64_t *bar, ui
 {
     if (sm.abort_flag)
         return false;
-    if (mbar_wait(bar, parity))
+    if (mbar_wait(bar, parity, sm.wait_limit))
         return true;
     set_flag(flags, kDevTimeout);
     set_flag(flags + 1, site);
@@ -168,7 +169,7 @@ __device__ __forceinline__ bool wait_tag(SimtSmem<D> &sm, int stage, uint32_t T,
     while (sm.stage_tile[stage] != T) {
         if (sm.abort_flag)
             return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > sm.wait_limit) {
             set_flag(flags, kDevTimeout);
             set_flag(flags + 1, kWaitTag);
             sm.abort_flag = 1;
@@ -305,16 +306,18 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
         cur = ahead;
         ++j;
     }
-    if (sm.abort_flag) {
-        // Let every copy this CTA started land before the CTA can exit.
+    {
+        // Let every copy this CTA started land before the CTA can exit.  On
+        // the normal path every tile and query copy was consumed and these
+        // phases are complete; after a consumer gave up, some may not be.
         const uint32_t n = T < (uint32_t)NSTAGE ? T : (uint32_t)NSTAGE;
         for (uint32_t k = 1; k <= n; ++k) {
             const uint32_t t = T - k;
-            (void)mbar_wait(&sm.full[t % NSTAGE], (t / NSTAGE) & 1u);
+            (void)mbar_wait(&sm.full[t % NSTAGE], (t / NSTAGE) & 1u, sm.wait_limit);
         }
         for (uint32_t k = 1; k <= 2 && k <= q_issued; ++k) {
             const uint32_t jj = q_issued - k;  // the last two query copies started
-            (void)mbar_wait(&sm.q_full[jj & 1], (jj >> 1) & 1u);
+            (void)mbar_wait(&sm.q_full[jj & 1], (jj >> 1) & 1u, sm.wait_limit);
         }
     }
 }
@@ -412,9 +415,12 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
         for (; t < ntiles; t += NCW) {
             const uint32_t T = T0 + t;
             const int stage = T % NSTAGE;
-            const bool ok = wait_tag<D>(sm, stage, T, p.flags) &&
-                            wait_or_abort(sm, &sm.full[stage], (T / NSTAGE) & 1u, p.flags, kWaitFull);
-            __syncwarp();
+            // the warp takes one decision: a lane whose wait ran out makes
+            // every lane skip the tile (the CTA is winding down then)
+            const bool ok = __all_sync(
+                0xffffffffu, wait_tag<D>(sm, stage, T, p.flags) &&
+                                 wait_or_abort(sm, &sm.full[stage], (T / NSTAGE) & 1u, p.flags,
+                                               kWaitFull));
             if (!ok)
                 continue;
             const uint8_t *Ks = sm.kv[stage][0];
@@ -562,7 +568,8 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                     pv_step(kk);
             }
             __syncwarp();
-            if (lane == 0)
+            // (the test switch: every CTA withholds the release of its first tile)
+            if (lane == 0 && !(p.withhold && T == 0))
                 mbar_arrive(&sm.empty[stage]);
         }
         T0 += ntiles;
@@ -697,6 +704,7 @@ __global__ void __launch_bounds__(simt_threads<D>(), 1)
         mbar_init(&sm.w_free, 1);
         sm.w_count = 0;
         sm.abort_flag = 0;
+        sm.wait_limit = p.wait_limit;
         fence_mbar_init();
     }
     wait_prior_grid();

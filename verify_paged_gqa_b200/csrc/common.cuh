@@ -25,7 +25,9 @@ constexpr int kMaxDevices = 64;
 // A pipeline wait gives up after this many SM clock cycles (about two
 // seconds at B200 clocks; an internal error: every wait in these kernels is
 // satisfied by work issued earlier in the same CTA).  The SM's own cycle
-// counter is used because it only moves forward.
+// counter is used because it only moves forward.  A call carries its limit
+// in AttnParams::wait_limit (this value unless a test asks for a shorter
+// one).
 constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // Word 1 of the workspace header records which wait gave up (one bit per
@@ -54,6 +56,13 @@ struct AttnParams {
     int32_t VT;                 // entry tiles of work in front of every unit
     int32_t whole;              // 1: CTA c takes unit c whole (no split, no partials)
     int32_t has_tree;           // 1: tree-verify call (the tree pointer holds the masks)
+    // Test switch (0 in every library call): 1 makes CTA 0 withhold one
+    // synchronous arrival that no copy or MMA completes -- the softmax warps'
+    // P-ready arrival of their first tile (tensor-core kernels), or the
+    // consumer's release of the first ring stage (CUDA-core kernel) -- so
+    // that a bounded wait runs out and the failure path runs.
+    int32_t withhold;
+    long long wait_limit;       // cycles a pipeline wait may take (kWaitLimitCycles)
     long long *first_tile;      // workspace: where each stream's work starts in the launch
     long long *total_tiles;     // workspace: work tiles of the launch
     float scale_log2;           // scale * log2(e): scores are kept in log2 units
@@ -132,7 +141,8 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
 // Waits for the phase with the given parity to complete; false after the
 // time limit (the caller records kDevTimeout and winds down).  A phase that
 // has already completed costs one non-blocking test.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          long long limit = kWaitLimitCycles)
 {
     if (mbar_test_wait(bar, parity))
         return true;
@@ -142,7 +152,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((it & 255u) == 0 && clock64() - t0 > kWaitLimitCycles)
+        if ((it & 255u) == 0 && clock64() - t0 > limit)
             return false;
     }
 }

@@ -27,7 +27,7 @@ __device__ __forceinline__ bool pwait(Sm &sm, uint64_t *bar, uint32_t parity, ui
 {
     if (sm.abort_flag)
         return false;
-    if (mbar_wait(bar, parity))
+    if (mbar_wait(bar, parity, sm.wait_limit))
         return true;
     set_flag(flags, kDevTimeout);
     set_flag(flags + 1, site);
@@ -107,12 +107,14 @@ __device__ __forceinline__ void ring_producer(const AttnParams &p, const CUtenso
             pg1 = pg2;
         }
     }
-    if (!ok || sm.abort_flag) {
-        // let the copies in flight land before the CTA exits
+    {
+        // Let the copies in flight land before the CTA can exit.  On the
+        // normal path every unit was consumed and these phases are complete;
+        // after another role gave up, some may still be in flight.
         const uint32_t nf = U < (uint32_t)NU ? U : (uint32_t)NU;
         for (uint32_t k = 1; k <= nf; ++k) {
             const uint32_t v = U - k;
-            (void)mbar_wait(&sm.full[v % NU], (v / NU) & 1u);
+            (void)mbar_wait(&sm.full[v % NU], (v / NU) & 1u, p.wait_limit);
         }
     }
 }

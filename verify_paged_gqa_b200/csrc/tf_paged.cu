@@ -5,6 +5,7 @@
 // depends only on host arguments and the device's SM count, so a captured
 // graph stays valid while lens grow up to max_len.
 #include "../../include/tf_paged.h"
+#include "../../include/tf_paged_testing.h"
 #include "launch.cuh"
 #include "plan.cuh"
 
@@ -122,6 +123,8 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     p.W = rows;
     p.M = static_cast<int32_t>(M);
     p.has_tree = tree ? 1 : 0;
+    p.withhold = 0;
+    p.wait_limit = kWaitLimitCycles;
     // Rows sharing a KV head go to the tensor cores as a dense QK^T / PV
     // tile: up to 64 rows (any count at head dims 256 and 512, in blocks of
     // 32) with the positions on the MMA's M, larger blocks with the rows
@@ -187,14 +190,22 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     return TF_OK;
 }
 
+// The test hooks of one call (tf_testing_paged_attn); none in library calls.
+struct Faults {
+    long long wait_limit = kWaitLimitCycles;
+    int32_t withhold = 0;
+};
+
 int attn_call(const tf_kv_pool *pool, const tf_streams *st, const void *q, int32_t Hq,
               int32_t rows, int32_t rows_max, const uint8_t *tree, float scale, float *out,
-              void *ws, size_t ws_bytes, void *stream)
+              void *ws, size_t ws_bytes, void *stream, const Faults &faults = Faults{})
 {
     Plan plan;
     int rc = make_plan(pool, st, Hq, rows, rows_max, tree != nullptr, &plan);
     if (rc != TF_OK)
         return rc;
+    plan.p.wait_limit = faults.wait_limit;
+    plan.p.withhold = faults.withhold;
     if (!std::isfinite(scale))
         return TF_EINVAL;
     if (st->n_streams == 0)
@@ -373,6 +384,22 @@ int tf_paged_attn_prompt(const tf_kv_pool *pool, const tf_streams *streams, cons
 {
     return attn_call(pool, streams, q, n_q_heads, rows, 4096, nullptr, scale, out, workspace,
                      workspace_bytes, stream);
+}
+
+int tf_testing_paged_attn(const tf_kv_pool *pool, const tf_streams *streams, const void *q,
+                          int32_t n_q_heads, int32_t rows, float scale, float *out,
+                          void *workspace, size_t workspace_bytes, int64_t wait_limit_cycles,
+                          int32_t withhold, void *stream)
+{
+    if (wait_limit_cycles < 1000000 || wait_limit_cycles > kWaitLimitCycles)
+        return TF_EINVAL;
+    if (withhold != 0 && withhold != 1)
+        return TF_EINVAL;
+    Faults f;
+    f.wait_limit = wait_limit_cycles;
+    f.withhold = withhold;
+    return attn_call(pool, streams, q, n_q_heads, rows, 4096, nullptr, scale, out, workspace,
+                     workspace_bytes, stream, f);
 }
 
 int tf_workspace_status(void *workspace, uint32_t *flags, void *stream)
