@@ -5,8 +5,9 @@ Every pipeline wait in the attention kernels is bounded.  The test hook
 tf_testing_paged_attn (include/tf_paged_testing.h) gives a call a short wait
 limit (about 10 ms) and makes CTA 0 withhold one arrival that no copy or MMA
 completes: the softmax warps' "P is written" arrival of their first tile on
-the tensor-core kernels, the release of the first ring stage on the CUDA-core
-kernel.  The wait on it must run out: the call returns, its status word holds
+the tensor-core kernels (whose ring is filled by TMA, or gathered row by row
+for pages that are not a multiple of 128), the release of the first ring
+stage on the CUDA-core kernel.  The wait on it must run out: the call returns, its status word holds
 TF_DEV_TIMEOUT and a wait-site bit, and the next ordinary call on the same
 stream and workspace matches the oracle with a clean status word.
 """
@@ -29,7 +30,9 @@ SHORT_LIMIT = 20_000_000   # SM cycles: about 10 ms at B200 clocks
     ("verify, position-major kernel (64-row blocks)", 128, 8, 512, 8, [60000, 3000]),
     ("head dim 512 verify, position-major kernel (one issuer)", 512, 8, 512, 4, [30000, 3000]),
     ("prompt chunk, row-major kernel", 128, 4, 512, 200, [60000, 3000]),
-    ("pages of 64, CUDA-core kernel", 128, 4, 64, 1, [200000, 3000]),
+    ("pages of 64, position-major kernel (tiles gathered across pages)", 128, 4, 64, 1,
+     [60000, 3000]),
+    ("head dim 512 decode, CUDA-core kernel", 512, 4, 512, 1, [60000, 3000]),
 ])
 def test_a_withheld_arrival_times_out_and_the_next_call_is_clean(name, d, G, P, W, lens):
     import verify_paged_gqa_b200 as tf

@@ -270,15 +270,34 @@ def test_parity_gqa16_hd512(W):
     run_parity(w, [5000, 700, W], W)
 
 
-def test_hd256_needs_pages_of_128():
-    import verify_paged_gqa_b200 as tf
-    w = small_workload(256, 4, 64, 1, seed=9700)
-    case = synth.make_case(w, lens=[300])
-    dc = DeviceCase(case)
-    ws = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
-    with pytest.raises(tf.TFError) as e:
-        dc.attend(ws=ws)
-    assert e.value.status == tf.TF_EUNSUPPORTED
+@pytest.mark.parametrize("P", [64, 37, 1, 100])
+@pytest.mark.parametrize("W", [1, 4])
+def test_hd256_any_page_size(P, W):
+    """Head dim 256 over pages that are not a multiple of 128: the tiles that
+    straddle pages are gathered row by row."""
+    w = small_workload(256, 4, P, W, seed=9700 + P + W)
+    lens = [P * 5 + 3, W + 1, 700] if P > 1 else [300, W + 1, 129]
+    run_parity(w, lens, W)
+
+
+@pytest.mark.parametrize("d,G,W", [(128, 4, 1), (128, 8, 8), (256, 8, 4), (512, 8, 4),
+                                   (512, 4, 1), (128, 4, 100)])
+def test_page_size_changes_no_output_bit(d, G, W):
+    """The same streams in pools of pages of 512, 128, 37 and 1 positions:
+    whole TMA boxes or rows gathered across pages, the outputs are equal byte
+    for byte (the arithmetic depends on positions, never on the pages)."""
+    lens = [1300, W + 2, 777]
+    outs = []
+    for P in (512, 128, 37, 1):
+        w = small_workload(d, G, P, W, seed=9800 + d + G + W)   # same seed: same K, V, q
+        case = synth.make_case(w, lens=lens, rows=W)
+        outs.append(DeviceCase(case).attend())
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
+    ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, W, w.group, w.scale,
+                        threads=8)
+    assert max_abs(outs[0], ref) <= TOL
 
 
 # --- tree-mask verify: each window row sees the positions before the window
@@ -428,14 +447,27 @@ def test_page37_bad_page_is_flagged_and_shapes_refused():
     dc.table[0, 3] = dc.k_pool.shape[0] + 2      # a page in the middle of a straddling tile
     dc.attend(ws=ws)
     assert tf.tf_workspace_status(ws) & tf.TF_DEV_BAD_PAGE
-    # head dim 256 (with or without tree masks) needs pages that are a multiple of 128
+    # a page id past the pool on the tensor-core kernels' gathered tiles
+    for d, W in ((128, 8), (256, 4), (512, 4)):
+        w3 = small_workload(d, 8, 37, W, seed=11303 + d)
+        dc3 = DeviceCase(synth.make_case(w3, lens=[900, 300], rows=W))
+        ws3 = dc3.workspace(W)
+        tf.tf_workspace_status(ws3)
+        dc3.table[1, 2] = -7
+        out = dc3.attend(ws=ws3)
+        assert tf.tf_workspace_status(ws3) & tf.TF_DEV_BAD_PAGE
+        ref = oracle.attend(dc3.case.q[:1], dc3.case.k_lin[:1], dc3.case.v_lin[:1],
+                            dc3.case.lens[:1], W, 8, w3.scale)
+        assert max_abs(out[:1], ref) <= TOL              # the other stream is untouched
+    # head dim 256 over pages of 37, with and without tree masks
     w2 = small_workload(256, 4, 37, 4, seed=11301)
-    dc2 = DeviceCase(synth.make_case(w2, lens=[300], rows=4))
-    ws2 = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
-    for tree in (None, synth.tree_masks((11302,), 1, 4)):
-        with pytest.raises(tf.TFError) as e:
-            dc2.attend(ws=ws2, tree=tree)
-        assert e.value.status == tf.TF_EUNSUPPORTED
+    case2 = synth.make_case(w2, lens=[300, 41], rows=4)
+    dc2 = DeviceCase(case2)
+    for tree in (None, synth.tree_masks((11302,), 2, 4)):
+        out = dc2.attend(tree=tree)
+        ref = oracle.attend(case2.q, case2.k_lin, case2.v_lin, case2.lens, 4, 4, w2.scale,
+                            threads=8, tree=tree)
+        assert max_abs(out, ref) <= TOL
 
 
 # --- the state copy: a stream's K/V walked from one set of pages to another

@@ -175,8 +175,9 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, float (&x)[NR])
 
 // ---- MMA issuer --------------------------------------------------------------
 
-// S^T = K Q^T for one tile: DB units, 8 MMAs (K = 16 dims) each.
-template <int D, int NR>
+// S^T = K Q^T for one tile: DB units, 8 MMAs (K = 16 dims) each.  Gathered
+// units (kG) were written through the generic proxy: fence before the MMAs.
+template <int D, int NR, bool kG>
 __device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d_tmem,
                                       uint32_t ring0, uint32_t q0, uint32_t *flags)
 {
@@ -191,6 +192,8 @@ __device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d
         if (!pwait(sm, &sm.full[st], (U / NRING) & 1u, flags, kWaitFull))
             return false;
         tc_fence_after();
+        if constexpr (kG)
+            fence_async_smem();
         const uint32_t ka = ring0 + st * kUnit;
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
@@ -205,7 +208,7 @@ __device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d
     return true;
 }
 
-template <int D, int NR>
+template <int D, int NR, bool kG>
 __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
 {
     using C = PmCfg<D, NR>;
@@ -225,7 +228,7 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         ok = pwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
         tc_fence_after();
-        ok = ok && pm_qk(sm, U, tmem + C::kColS + (T0 & 1u) * NR, ring0, q0, p.flags);
+        ok = ok && pm_qk<D, NR, kG>(sm, U, tmem + C::kColS + (T0 & 1u) * NR, ring0, q0, p.flags);
         if (!ok)
             break;
         umma_commit(&sm.s_full[T0 & 1u]);
@@ -234,7 +237,8 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
         for (int t = 0; t < n; ++t) {
             const uint32_t T = T0 + t;
             if (t + 1 < n) {
-                ok = pm_qk(sm, U, tmem + C::kColS + ((T + 1) & 1u) * NR, ring0, q0, p.flags);
+                ok = pm_qk<D, NR, kG>(sm, U, tmem + C::kColS + ((T + 1) & 1u) * NR, ring0, q0,
+                                      p.flags);
                 if (!ok)
                     break;
                 umma_commit(&sm.s_full[(T + 1) & 1u]);
@@ -253,6 +257,8 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
                 tc_fence_after();
                 if (!ok)
                     break;
+                if constexpr (kG)
+                    fence_async_smem();
                 const uint32_t va = ring0 + st * kUnit;
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
@@ -361,9 +367,65 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
     }
 }
 
+// The whole producer warp: the unit order of pm_producer_dual, gathered row by
+// row (page sizes that are not a multiple of 128; ring.cuh).
+template <int D, int NR>
+__device__ __forceinline__ void pm_producer_dual_gather(const PmArgs &a, PmSmem<D, NR> &sm,
+                                                        int lane)
+{
+    using C = PmCfg<D, NR>;
+    const AttnParams &p = a.p;
+    const uint64_t pol = l2_evict_first_policy();
+    uint32_t UK = 0, UV = 0;  // units issued
+    bool ok = true;
+    SegCursor cur;
+    cur.init(p, sm.range);
+    WorkItem it;
+    while (ok && cur.next(p, it)) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
+        const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
+        TileRows r0 = tile_rows(p, trow, it.kh, it.key0, it.len, lane);
+#pragma unroll 1
+        for (int kb = 0; ok && kb < C::DB; ++kb) {
+            ok = gather_unit(p, sm, (int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, p.k_pool, r0, kb,
+                             lane, pol);
+            UK += ok ? 1u : 0u;
+        }
+        for (int t = 0; ok && t < n; ++t) {
+            const int pos = it.key0 + t * PT;
+            TileRows r1 = r0;
+            if (t + 1 < n)
+                r1 = tile_rows(p, trow, it.kh, pos + PT, it.len, lane);
+#pragma unroll 1
+            for (int kb = 0; ok && kb < C::DB; ++kb) {
+                if (t + 1 < n) {
+                    ok = gather_unit(p, sm, (int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, p.k_pool,
+                                     r1, kb, lane, pol);
+                    UK += ok ? 1u : 0u;
+                }
+                if (ok) {
+                    ok = gather_unit(p, sm, C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u,
+                                     p.v_pool, r0, kb, lane, pol);
+                    UV += ok ? 1u : 0u;
+                }
+            }
+            r0 = r1;
+        }
+    }
+    if (lane == 0) {
+        // let the copies in flight land before the CTA can exit
+        for (uint32_t k = 1; k <= (UK < (uint32_t)C::NK ? UK : (uint32_t)C::NK); ++k)
+            (void)mbar_wait(&sm.full[(UK - k) % C::NK], ((UK - k) / C::NK) & 1u, sm.wait_limit);
+        for (uint32_t k = 1; k <= (UV < (uint32_t)C::NV ? UV : (uint32_t)C::NV); ++k)
+            (void)mbar_wait(&sm.full[C::NK + (UV - k) % C::NV], ((UV - k) / C::NV) & 1u,
+                            sm.wait_limit);
+    }
+    __syncwarp();
+}
+
 // One lane: S^T(T) = K Q^T into S^T buffer T % 2 once the softmax arrived on
 // p_full for tile T - 2 (it is done reading that buffer then).
-template <int D, int NR>
+template <int D, int NR, bool kG>
 __device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
 {
     using C = PmCfg<D, NR>;
@@ -383,7 +445,7 @@ __device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
             if (T >= 2)
                 ok = pwait(sm, &sm.p_full[T & 1u], ((T - 2) >> 1) & 1u, p.flags, kWaitQEmpty);
             tc_fence_after();
-            ok = ok && pm_qk(sm, U, tmem + C::kColS + (T & 1u) * NR, ring0, q0, p.flags);
+            ok = ok && pm_qk<D, NR, kG>(sm, U, tmem + C::kColS + (T & 1u) * NR, ring0, q0, p.flags);
             if (!ok)
                 break;
             umma_commit(&sm.s_full[T & 1u]);
@@ -400,7 +462,7 @@ __device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
 // P^T(T).  Before the PV of a stream's last tile the warp zeroes the V rows
 // past the stream's end (their P is 0, but 0 * NaN = NaN); it is the V
 // part's only consumer, so its wait on the slot names the right phase.
-template <int D, int NR>
+template <int D, int NR, bool kG>
 __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm, int lane)
 {
     using C = PmCfg<D, NR>;
@@ -443,6 +505,8 @@ __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm,
             }
             if (lane == 0) {
                 tc_fence_after();
+                if constexpr (kG)
+                    fence_async_smem();
                 const uint32_t va = smem_addr(sm.ring[st]);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
@@ -796,7 +860,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
     }
 }
 
-template <int D, int NR, bool kTree>
+template <int D, int NR, bool kTree, bool kG>
 __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     attn_pm_kernel(const __grid_constant__ PmArgs a)
 {
@@ -809,7 +873,8 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NU; ++s) {
-            mbar_init(&sm.full[s], 1);
+            // a gathered unit completes with one arrival per producer lane
+            mbar_init(&sm.full[s], kG ? 32 : 1);
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.q_full, 1);
@@ -839,23 +904,30 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     tc_fence_after();
 
     if (warp == 0) {
-        if (lane == 0) {
+        if constexpr (kG) {
             if constexpr (C::kDual)
-                pm_producer_dual<D, NR>(a, sm);
+                pm_producer_dual_gather<D, NR>(a, sm, lane);
             else
-                ring_producer<C::DB, C::NU>(a.p, &a.kmap, &a.vmap, sm);
+                ring_producer_gather<C::DB, C::NU>(a.p, sm, lane);
+        } else {
+            if (lane == 0) {
+                if constexpr (C::kDual)
+                    pm_producer_dual<D, NR>(a, sm);
+                else
+                    ring_producer<C::DB, C::NU>(a.p, &a.kmap, &a.vmap, sm);
+            }
+            __syncwarp();
         }
-        __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             if constexpr (C::kDual)
-                pm_qk_issuer<D, NR>(a, sm);
+                pm_qk_issuer<D, NR, kG>(a, sm);
             else
-                pm_issuer<D, NR>(a, sm);
+                pm_issuer<D, NR, kG>(a, sm);
         }
         __syncwarp();
     } else if (C::kDual && warp == C::kPvWarp) {
-        pm_pv_issuer<D, NR>(a, sm, lane);
+        pm_pv_issuer<D, NR, kG>(a, sm, lane);
     } else {
         pm_softmax<D, NR, kTree>(a, sm, warp, lane);
     }
@@ -869,7 +941,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     }
 }
 
-template <int D, int NR, bool kTree>
+template <int D, int NR, bool kTree, bool kG>
 cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
 {
     PmArgs a;
@@ -878,22 +950,23 @@ cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
         return cudaErrorInvalidValue;
     static std::atomic<bool> configured[kMaxDevices];
     constexpr size_t bytes = pm_smem_bytes<D, NR>();
-    const cudaError_t e = set_smem_limit_once(attn_pm_kernel<D, NR, kTree>, bytes, configured);
+    const cudaError_t e = set_smem_limit_once(attn_pm_kernel<D, NR, kTree, kG>, bytes, configured);
     if (e != cudaSuccess)
         return e;
-    return launch_dependent(attn_pm_kernel<D, NR, kTree>, dim3(grid), dim3(PmCfg<D, NR>::kThreads),
-                            bytes, stream, a);
+    return launch_dependent(attn_pm_kernel<D, NR, kTree, kG>, dim3(grid),
+                            dim3(PmCfg<D, NR>::kThreads), bytes, stream, a);
 }
 
 }  // namespace
 
-// Rows per row block, or 0 when this kernel does not take the call: tiles
-// stay inside a page, and causal blocks of more than 64 rows at head dim 128
-// go to the row-major tensor-core kernel (tree calls run here with several
-// row blocks).
+// Rows per row block, or 0 when this kernel does not take the call: causal
+// blocks of more than 64 rows at head dim 128 go to the row-major tensor-core
+// kernel (tree calls run here with several row blocks), and pool rows are
+// addressed by 32-bit coordinates.  Any page size: tiles that straddle pages
+// are gathered row by row.
 int pm_rows(const AttnParams &p)
 {
-    if (p.P % PT != 0 || !pool_rows_fit(p))
+    if (!pool_rows_fit(p))
         return 0;
     if (p.D == 128)
         return p.M <= 32 ? 32 : (p.M <= 64 || p.has_tree) ? 64 : 0;
@@ -902,24 +975,30 @@ int pm_rows(const AttnParams &p)
     return 0;
 }
 
-template <bool kTree>
+template <bool kTree, bool kG>
 cudaError_t launch_attn_pm_t(const AttnParams &p, int grid, cudaStream_t stream)
 {
     if (p.D == 128 && p.RB == 32)
-        return launch_pm<128, 32, kTree>(p, grid, stream);
+        return launch_pm<128, 32, kTree, kG>(p, grid, stream);
     if (p.D == 128 && p.RB == 64)
-        return launch_pm<128, 64, kTree>(p, grid, stream);
+        return launch_pm<128, 64, kTree, kG>(p, grid, stream);
     if (p.D == 256 && p.RB == 32)
-        return launch_pm<256, 32, kTree>(p, grid, stream);
+        return launch_pm<256, 32, kTree, kG>(p, grid, stream);
     if (p.D == 512 && p.RB == 32)
-        return launch_pm<512, 32, kTree>(p, grid, stream);
+        return launch_pm<512, 32, kTree, kG>(p, grid, stream);
     return cudaErrorInvalidValue;
 }
 
+// Pages that are a multiple of 128 positions hold whole tiles (TMA boxes);
+// any other page size is gathered.
 cudaError_t launch_attn_pm(const AttnParams &p, int grid, cudaStream_t stream)
 {
-    return p.has_tree ? launch_attn_pm_t<true>(p, grid, stream)
-                      : launch_attn_pm_t<false>(p, grid, stream);
+    const bool gather = p.P % PT != 0;
+    if (p.has_tree)
+        return gather ? launch_attn_pm_t<true, true>(p, grid, stream)
+                      : launch_attn_pm_t<true, false>(p, grid, stream);
+    return gather ? launch_attn_pm_t<false, true>(p, grid, stream)
+                  : launch_attn_pm_t<false, false>(p, grid, stream);
 }
 
 }  // namespace tfp

@@ -90,7 +90,9 @@ struct PrArgs {
 
 // S(u) = Q K^T for tile u of the CTA: the K unit's 8 MMAs (K = 16 dims each),
 // A (Q) read from tensor memory.  S has one buffer: it is free once the
-// softmax warps read S(u - 1).
+// softmax warps read S(u - 1).  Gathered units (kG) were written through the
+// generic proxy: fence before the MMAs.
+template <bool kG>
 __device__ __forceinline__ bool pr_qk(PrSmem &sm, uint32_t &U, uint32_t u, uint32_t tmem,
                                       uint32_t ring0, uint32_t *flags)
 {
@@ -101,6 +103,8 @@ __device__ __forceinline__ bool pr_qk(PrSmem &sm, uint32_t &U, uint32_t u, uint3
     if (!pwait(sm, &sm.full[st], (U / NU) & 1u, flags, kWaitFull))
         return false;
     tc_fence_after();
+    if constexpr (kG)
+        fence_async_smem();
     const uint32_t ka = ring0 + st * kRingUnit;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
@@ -115,6 +119,7 @@ __device__ __forceinline__ bool pr_qk(PrSmem &sm, uint32_t &U, uint32_t u, uint3
 }
 
 // One lane.  Per segment: QK(0), then per tile t: QK(t + 1), PV(t).
+template <bool kG>
 __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
 {
     const AttnParams &p = a.p;
@@ -134,7 +139,7 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         ok = pwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
         tc_fence_after();
-        ok = ok && pr_qk(sm, U, T0, tmem, ring0, p.flags);
+        ok = ok && pr_qk<kG>(sm, U, T0, tmem, ring0, p.flags);
         if (!ok)
             break;
         if (n == 1)
@@ -142,7 +147,7 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
         for (int t = 0; t < n; ++t) {
             const uint32_t T = T0 + t;
             if (t + 1 < n) {
-                ok = pr_qk(sm, U, T + 1, tmem, ring0, p.flags);
+                ok = pr_qk<kG>(sm, U, T + 1, tmem, ring0, p.flags);
                 if (!ok)
                     break;
                 if (t + 2 == n)
@@ -157,6 +162,8 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
             tc_fence_after();
             if (!ok)
                 break;
+            if constexpr (kG)
+                fence_async_smem();
             const uint32_t va = ring0 + st * kRingUnit;
 #pragma unroll
             for (int s = 0; s < 8; ++s)
@@ -420,6 +427,7 @@ __device__ __forceinline__ void pr_softmax(const PrArgs &a, PrSmem &sm, int warp
     }
 }
 
+template <bool kG>
 __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_constant__ PrArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -430,7 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NU; ++s) {
-            mbar_init(&sm.full[s], 1);
+            // a gathered unit completes with one arrival per producer lane
+            mbar_init(&sm.full[s], kG ? 32 : 1);
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.q_full, 8);
@@ -458,12 +467,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
     tc_fence_after();
 
     if (warp == 0) {
-        if (lane == 0)
-            ring_producer<1, NU>(a.p, &a.kmap, &a.vmap, sm);
-        __syncwarp();
+        if constexpr (kG) {
+            ring_producer_gather<1, NU>(a.p, sm, lane);
+        } else {
+            if (lane == 0)
+                ring_producer<1, NU>(a.p, &a.kmap, &a.vmap, sm);
+            __syncwarp();
+        }
     } else if (warp == 1) {
         if (lane == 0)
-            pr_issuer(a, sm);
+            pr_issuer<kG>(a, sm);
         __syncwarp();
     } else {
         pr_softmax(a, sm, warp, lane);
@@ -483,10 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
 // Rows per row block of this kernel.
 int prompt_rows() { return RR; }
 
-// Tiles stay inside a page; pool rows are addressed by 32-bit TMA coordinates.
+// Pool rows are addressed by 32-bit coordinates.  Any page size: tiles that
+// straddle pages are gathered row by row.
 bool prompt_supported(const AttnParams &p)
 {
-    return p.D == DD && p.P % PT == 0 && pool_rows_fit(p);
+    return p.D == DD && pool_rows_fit(p);
 }
 
 cudaError_t launch_attn_prompt(const AttnParams &p, int grid, cudaStream_t stream)
@@ -495,11 +509,22 @@ cudaError_t launch_attn_prompt(const AttnParams &p, int grid, cudaStream_t strea
     a.p = p;
     if (!make_pool_map(&a.kmap, p.k_pool, p, PT) || !make_pool_map(&a.vmap, p.v_pool, p, PT))
         return cudaErrorInvalidValue;
+    // pages that are a multiple of 128 positions hold whole tiles (TMA boxes);
+    // any other page size is gathered
+    if (p.P % PT != 0) {
+        static std::atomic<bool> configured[kMaxDevices];
+        const cudaError_t e = set_smem_limit_once(attn_prompt_kernel<true>, kPrSmemBytes, configured);
+        if (e != cudaSuccess)
+            return e;
+        return launch_dependent(attn_prompt_kernel<true>, dim3(grid), dim3(kThreads), kPrSmemBytes,
+                                stream, a);
+    }
     static std::atomic<bool> configured[kMaxDevices];
-    const cudaError_t e = set_smem_limit_once(attn_prompt_kernel, kPrSmemBytes, configured);
+    const cudaError_t e = set_smem_limit_once(attn_prompt_kernel<false>, kPrSmemBytes, configured);
     if (e != cudaSuccess)
         return e;
-    return launch_dependent(attn_prompt_kernel, dim3(grid), dim3(kThreads), kPrSmemBytes, stream, a);
+    return launch_dependent(attn_prompt_kernel<false>, dim3(grid), dim3(kThreads), kPrSmemBytes,
+                            stream, a);
 }
 
 }  // namespace tfp

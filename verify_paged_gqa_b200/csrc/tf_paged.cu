@@ -132,13 +132,14 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     // too (decode at GQA 4): its two MMA issuers keep pace with HBM at any
     // clock, where the CUDA-core kernel's FMAs fall behind under the power
     // cap (12 x 40,960 decode: 341 -> 296 us per call).  Head dim 512 keeps
-    // such calls on the CUDA-core kernel, and so do pages whose size is not
-    // a multiple of 128.
+    // such calls on the CUDA-core kernel.  Any page size runs on the
+    // tensor-core kernels (tiles that straddle pages are gathered row by
+    // row); only pools past 2^31 rows fall back to the CUDA-core kernel.
     plan->kernel = Kernel::kSimt;
     p.RB = kSimtRows;
     if (tree) {
         // tree masks: the position-major kernel (any row count), else the
-        // CUDA-core kernel (page sizes that are not a multiple of 128)
+        // CUDA-core kernel (pools past 2^31 rows)
         const int nr = pm_rows(p);
         if (nr > 0) {
             plan->kernel = Kernel::kPm;
