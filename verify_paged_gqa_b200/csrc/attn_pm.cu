@@ -129,10 +129,13 @@ static_assert(pm_smem_bytes<128, 64>() <= kSmemCap, "smem");
 static_assert(pm_smem_bytes<256, 32>() <= kSmemCap, "smem");
 static_assert(pm_smem_bytes<512, 32>() <= kSmemCap, "smem");
 
+// Kernel arguments: the call's parameters and the K and V pools' tensor maps
+// (one 128-row box, or for tiles assembled from pages one map per box height).
+template <bool kG>
 struct PmArgs {
     AttnParams p;
-    CUtensorMap kmap;
-    CUtensorMap vmap;
+    CUtensorMap kmap[kG ? kBoxHeights : 1];
+    CUtensorMap vmap[kG ? kBoxHeights : 1];
 };
 
 // Reduces v[i] (one value per row, N rows) across the warp: lane l ends up
@@ -175,9 +178,8 @@ __device__ __forceinline__ void load_scores(uint32_t taddr, float (&x)[NR])
 
 // ---- MMA issuer --------------------------------------------------------------
 
-// S^T = K Q^T for one tile: DB units, 8 MMAs (K = 16 dims) each.  Gathered
-// units (kG) were written through the generic proxy: fence before the MMAs.
-template <int D, int NR, bool kG>
+// S^T = K Q^T for one tile: DB units, 8 MMAs (K = 16 dims) each.
+template <int D, int NR>
 __device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d_tmem,
                                       uint32_t ring0, uint32_t q0, uint32_t *flags)
 {
@@ -192,8 +194,6 @@ __device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d
         if (!pwait(sm, &sm.full[st], (U / NRING) & 1u, flags, kWaitFull))
             return false;
         tc_fence_after();
-        if constexpr (kG)
-            fence_async_smem();
         const uint32_t ka = ring0 + st * kUnit;
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
@@ -208,8 +208,8 @@ __device__ __forceinline__ bool pm_qk(PmSmem<D, NR> &sm, uint32_t &U, uint32_t d
     return true;
 }
 
-template <int D, int NR, bool kG>
-__device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
+template <int D, int NR, class A>
+__device__ __forceinline__ void pm_issuer(const A &a, PmSmem<D, NR> &sm)
 {
     using C = PmCfg<D, NR>;
     const AttnParams &p = a.p;
@@ -228,7 +228,7 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         ok = pwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
         tc_fence_after();
-        ok = ok && pm_qk<D, NR, kG>(sm, U, tmem + C::kColS + (T0 & 1u) * NR, ring0, q0, p.flags);
+        ok = ok && pm_qk(sm, U, tmem + C::kColS + (T0 & 1u) * NR, ring0, q0, p.flags);
         if (!ok)
             break;
         umma_commit(&sm.s_full[T0 & 1u]);
@@ -237,7 +237,7 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
         for (int t = 0; t < n; ++t) {
             const uint32_t T = T0 + t;
             if (t + 1 < n) {
-                ok = pm_qk<D, NR, kG>(sm, U, tmem + C::kColS + ((T + 1) & 1u) * NR, ring0, q0,
+                ok = pm_qk(sm, U, tmem + C::kColS + ((T + 1) & 1u) * NR, ring0, q0,
                                       p.flags);
                 if (!ok)
                     break;
@@ -257,8 +257,6 @@ __device__ __forceinline__ void pm_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
                 tc_fence_after();
                 if (!ok)
                     break;
-                if constexpr (kG)
-                    fence_async_smem();
                 const uint32_t va = ring0 + st * kUnit;
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
@@ -293,8 +291,8 @@ __device__ __forceinline__ bool pm_sees(int r, int rvis, uint32_t vis)
 // One lane: per segment the DB units of K(0), then per tile unit kb of
 // K(t + 1) (if any) and unit kb of V(t) in turn; K units into the ring's K
 // part, V units into its V part.  Page ids are read two tiles ahead.
-template <int D, int NR>
-__device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> &sm)
+template <int D, int NR, class A>
+__device__ __forceinline__ void pm_producer_dual(const A &a, PmSmem<D, NR> &sm)
 {
     using C = PmCfg<D, NR>;
     const AttnParams &p = a.p;
@@ -331,7 +329,7 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
         // (UK and UV count the units actually issued)
 #pragma unroll 1
         for (int kb = 0; ok && kb < C::DB; ++kb) {
-            ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg0, it.kh,
+            ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, a.kmap, pg0, it.kh,
                      it.key0 % p.P, kb);
             UK += ok ? 1u : 0u;
         }
@@ -341,12 +339,12 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
 #pragma unroll 1
             for (int kb = 0; ok && kb < C::DB; ++kb) {
                 if (t + 1 < n) {
-                    ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, &a.kmap, pg1, it.kh,
+                    ok = put((int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, a.kmap, pg1, it.kh,
                              (pos + PT) % p.P, kb);
                     UK += ok ? 1u : 0u;
                 }
                 if (ok) {
-                    ok = put(C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u, &a.vmap, pg0,
+                    ok = put(C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u, a.vmap, pg0,
                              it.kh, pos % p.P, kb);
                     UV += ok ? 1u : 0u;
                 }
@@ -367,11 +365,11 @@ __device__ __forceinline__ void pm_producer_dual(const PmArgs &a, PmSmem<D, NR> 
     }
 }
 
-// The whole producer warp: the unit order of pm_producer_dual, gathered row by
-// row (page sizes that are not a multiple of 128; ring.cuh).
-template <int D, int NR>
-__device__ __forceinline__ void pm_producer_dual_gather(const PmArgs &a, PmSmem<D, NR> &sm,
-                                                        int lane)
+// The whole producer warp: the unit order of pm_producer_dual, each unit
+// assembled from page pieces (page sizes that are not a multiple of 128;
+// ring.cuh).
+template <int D, int NR, class A>
+__device__ __forceinline__ void pm_producer_dual_pieces(const A &a, PmSmem<D, NR> &sm, int lane)
 {
     using C = PmCfg<D, NR>;
     const AttnParams &p = a.p;
@@ -384,32 +382,36 @@ __device__ __forceinline__ void pm_producer_dual_gather(const PmArgs &a, PmSmem<
     while (ok && cur.next(p, it)) {
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
-        TileRows r0 = tile_rows(p, trow, it.kh, it.key0, it.len, lane);
+        // rows and page ids of tiles t, t + 1 and t + 2 (the page ids are read
+        // two tiles before their first use)
+        auto nvalid = [&](int t) { return min(PT, it.len - (it.key0 + t * PT)); };
+        TilePages t0 = tile_pages(p, trow, it.key0, nvalid(0), lane);
+        TilePages t1 = n > 1 ? tile_pages(p, trow, it.key0 + PT, nvalid(1), lane) : t0;
 #pragma unroll 1
         for (int kb = 0; ok && kb < C::DB; ++kb) {
-            ok = gather_unit(p, sm, (int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, p.k_pool, r0, kb,
-                             lane, pol);
+            ok = pieces_unit(p, sm, (int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, a.kmap, t0, trow,
+                             it.kh, nvalid(0), kb, lane, pol);
             UK += ok ? 1u : 0u;
         }
         for (int t = 0; ok && t < n; ++t) {
             const int pos = it.key0 + t * PT;
-            TileRows r1 = r0;
-            if (t + 1 < n)
-                r1 = tile_rows(p, trow, it.kh, pos + PT, it.len, lane);
+            const TilePages t2 =
+                t + 2 < n ? tile_pages(p, trow, pos + 2 * PT, nvalid(t + 2), lane) : t1;
 #pragma unroll 1
             for (int kb = 0; ok && kb < C::DB; ++kb) {
                 if (t + 1 < n) {
-                    ok = gather_unit(p, sm, (int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, p.k_pool,
-                                     r1, kb, lane, pol);
+                    ok = pieces_unit(p, sm, (int)(UK % C::NK), ((UK / C::NK) & 1u) ^ 1u, a.kmap, t1,
+                                     trow, it.kh, nvalid(t + 1), kb, lane, pol);
                     UK += ok ? 1u : 0u;
                 }
                 if (ok) {
-                    ok = gather_unit(p, sm, C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u,
-                                     p.v_pool, r0, kb, lane, pol);
+                    ok = pieces_unit(p, sm, C::NK + (int)(UV % C::NV), ((UV / C::NV) & 1u) ^ 1u,
+                                     a.vmap, t0, trow, it.kh, nvalid(t), kb, lane, pol);
                     UV += ok ? 1u : 0u;
                 }
             }
-            r0 = r1;
+            t0 = t1;
+            t1 = t2;
         }
     }
     if (lane == 0) {
@@ -425,8 +427,8 @@ __device__ __forceinline__ void pm_producer_dual_gather(const PmArgs &a, PmSmem<
 
 // One lane: S^T(T) = K Q^T into S^T buffer T % 2 once the softmax arrived on
 // p_full for tile T - 2 (it is done reading that buffer then).
-template <int D, int NR, bool kG>
-__device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
+template <int D, int NR, class A>
+__device__ __forceinline__ void pm_qk_issuer(const A &a, PmSmem<D, NR> &sm)
 {
     using C = PmCfg<D, NR>;
     const AttnParams &p = a.p;
@@ -445,7 +447,7 @@ __device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
             if (T >= 2)
                 ok = pwait(sm, &sm.p_full[T & 1u], ((T - 2) >> 1) & 1u, p.flags, kWaitQEmpty);
             tc_fence_after();
-            ok = ok && pm_qk<D, NR, kG>(sm, U, tmem + C::kColS + (T & 1u) * NR, ring0, q0, p.flags);
+            ok = ok && pm_qk(sm, U, tmem + C::kColS + (T & 1u) * NR, ring0, q0, p.flags);
             if (!ok)
                 break;
             umma_commit(&sm.s_full[T & 1u]);
@@ -462,8 +464,8 @@ __device__ __forceinline__ void pm_qk_issuer(const PmArgs &a, PmSmem<D, NR> &sm)
 // P^T(T).  Before the PV of a stream's last tile the warp zeroes the V rows
 // past the stream's end (their P is 0, but 0 * NaN = NaN); it is the V
 // part's only consumer, so its wait on the slot names the right phase.
-template <int D, int NR, bool kG>
-__device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm, int lane)
+template <int D, int NR, class A>
+__device__ __forceinline__ void pm_pv_issuer(const A &a, PmSmem<D, NR> &sm, int lane)
 {
     using C = PmCfg<D, NR>;
     const AttnParams &p = a.p;
@@ -505,8 +507,6 @@ __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm,
             }
             if (lane == 0) {
                 tc_fence_after();
-                if constexpr (kG)
-                    fence_async_smem();
                 const uint32_t va = smem_addr(sm.ring[st]);
 #pragma unroll
                 for (int s = 0; s < 8; ++s)
@@ -531,8 +531,8 @@ __device__ __forceinline__ void pm_pv_issuer(const PmArgs &a, PmSmem<D, NR> &sm,
 // NW = 4 * NR / 32 softmax warps: warp w reads tensor-memory lanes
 // 32 * (w % 4) .. + 31 (tile positions, or O^T dims), and owns the 32 rows
 // [32 h, 32 h + 32) with h = (w - 2) / 4.
-template <int D, int NR, bool kTree>
-__device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, int warp, int lane)
+template <int D, int NR, bool kTree, class A>
+__device__ __forceinline__ void pm_softmax(const A &a, PmSmem<D, NR> &sm, int warp, int lane)
 {
     using C = PmCfg<D, NR>;
     constexpr int NT = C::kSoftThreads;
@@ -862,7 +862,7 @@ __device__ __forceinline__ void pm_softmax(const PmArgs &a, PmSmem<D, NR> &sm, i
 
 template <int D, int NR, bool kTree, bool kG>
 __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
-    attn_pm_kernel(const __grid_constant__ PmArgs a)
+    attn_pm_kernel(const __grid_constant__ PmArgs<kG> a)
 {
     using C = PmCfg<D, NR>;
     extern __shared__ uint8_t smem_raw[];
@@ -873,8 +873,7 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::NU; ++s) {
-            // a gathered unit completes with one arrival per producer lane
-            mbar_init(&sm.full[s], kG ? 32 : 1);
+            mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.q_full, 1);
@@ -906,28 +905,28 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
     if (warp == 0) {
         if constexpr (kG) {
             if constexpr (C::kDual)
-                pm_producer_dual_gather<D, NR>(a, sm, lane);
+                pm_producer_dual_pieces<D, NR>(a, sm, lane);
             else
-                ring_producer_gather<C::DB, C::NU>(a.p, sm, lane);
+                ring_producer_pieces<C::DB, C::NU>(a.p, a.kmap, a.vmap, sm, lane);
         } else {
             if (lane == 0) {
                 if constexpr (C::kDual)
                     pm_producer_dual<D, NR>(a, sm);
                 else
-                    ring_producer<C::DB, C::NU>(a.p, &a.kmap, &a.vmap, sm);
+                    ring_producer<C::DB, C::NU>(a.p, a.kmap, a.vmap, sm);
             }
             __syncwarp();
         }
     } else if (warp == 1) {
         if (lane == 0) {
             if constexpr (C::kDual)
-                pm_qk_issuer<D, NR, kG>(a, sm);
+                pm_qk_issuer<D, NR>(a, sm);
             else
-                pm_issuer<D, NR, kG>(a, sm);
+                pm_issuer<D, NR>(a, sm);
         }
         __syncwarp();
     } else if (C::kDual && warp == C::kPvWarp) {
-        pm_pv_issuer<D, NR, kG>(a, sm, lane);
+        pm_pv_issuer<D, NR>(a, sm, lane);
     } else {
         pm_softmax<D, NR, kTree>(a, sm, warp, lane);
     }
@@ -944,10 +943,16 @@ __global__ void __launch_bounds__(PmCfg<D, NR>::kThreads, 1)
 template <int D, int NR, bool kTree, bool kG>
 cudaError_t launch_pm(const AttnParams &p, int grid, cudaStream_t stream)
 {
-    PmArgs a;
+    PmArgs<kG> a;
     a.p = p;
-    if (!make_pool_map(&a.kmap, p.k_pool, p, PT) || !make_pool_map(&a.vmap, p.v_pool, p, PT))
-        return cudaErrorInvalidValue;
+    // one box of a whole 128-position tile, or boxes of 1, 2, 4, ..., 128 rows
+    // for tiles assembled from page pieces
+    for (int h = 0; h < (kG ? kBoxHeights : 1); ++h) {
+        const int rows = kG ? 1 << h : PT;
+        if (!make_pool_map(&a.kmap[h], p.k_pool, p, rows) ||
+            !make_pool_map(&a.vmap[h], p.v_pool, p, rows))
+            return cudaErrorInvalidValue;
+    }
     static std::atomic<bool> configured[kMaxDevices];
     constexpr size_t bytes = pm_smem_bytes<D, NR>();
     const cudaError_t e = set_smem_limit_once(attn_pm_kernel<D, NR, kTree, kG>, bytes, configured);

@@ -80,19 +80,20 @@ struct PrSmem {
 constexpr size_t kPrSmemBytes = sizeof(PrSmem) + 1024;  // + alignment slack
 static_assert(kPrSmemBytes <= 232448, "shared memory");
 
+// Kernel arguments: the call's parameters and the K and V pools' tensor maps
+// (one 128-row box, or for tiles assembled from pages one map per box height).
+template <bool kG>
 struct PrArgs {
     AttnParams p;
-    CUtensorMap kmap;
-    CUtensorMap vmap;
+    CUtensorMap kmap[kG ? kBoxHeights : 1];
+    CUtensorMap vmap[kG ? kBoxHeights : 1];
 };
 
 // ---- MMA issuer --------------------------------------------------------------
 
 // S(u) = Q K^T for tile u of the CTA: the K unit's 8 MMAs (K = 16 dims each),
 // A (Q) read from tensor memory.  S has one buffer: it is free once the
-// softmax warps read S(u - 1).  Gathered units (kG) were written through the
-// generic proxy: fence before the MMAs.
-template <bool kG>
+// softmax warps read S(u - 1).
 __device__ __forceinline__ bool pr_qk(PrSmem &sm, uint32_t &U, uint32_t u, uint32_t tmem,
                                       uint32_t ring0, uint32_t *flags)
 {
@@ -103,8 +104,6 @@ __device__ __forceinline__ bool pr_qk(PrSmem &sm, uint32_t &U, uint32_t u, uint3
     if (!pwait(sm, &sm.full[st], (U / NU) & 1u, flags, kWaitFull))
         return false;
     tc_fence_after();
-    if constexpr (kG)
-        fence_async_smem();
     const uint32_t ka = ring0 + st * kRingUnit;
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
@@ -119,8 +118,8 @@ __device__ __forceinline__ bool pr_qk(PrSmem &sm, uint32_t &U, uint32_t u, uint3
 }
 
 // One lane.  Per segment: QK(0), then per tile t: QK(t + 1), PV(t).
-template <bool kG>
-__device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
+template <class A>
+__device__ __forceinline__ void pr_issuer(const A &a, PrSmem &sm)
 {
     const AttnParams &p = a.p;
     const uint32_t tmem = sm.tmem_base;
@@ -139,7 +138,7 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
         const int n = (it.key1 - it.key0 + PT - 1) / PT;
         ok = pwait(sm, &sm.q_full, j & 1u, p.flags, kWaitQFull);
         tc_fence_after();
-        ok = ok && pr_qk<kG>(sm, U, T0, tmem, ring0, p.flags);
+        ok = ok && pr_qk(sm, U, T0, tmem, ring0, p.flags);
         if (!ok)
             break;
         if (n == 1)
@@ -147,7 +146,7 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
         for (int t = 0; t < n; ++t) {
             const uint32_t T = T0 + t;
             if (t + 1 < n) {
-                ok = pr_qk<kG>(sm, U, T + 1, tmem, ring0, p.flags);
+                ok = pr_qk(sm, U, T + 1, tmem, ring0, p.flags);
                 if (!ok)
                     break;
                 if (t + 2 == n)
@@ -162,8 +161,6 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
             tc_fence_after();
             if (!ok)
                 break;
-            if constexpr (kG)
-                fence_async_smem();
             const uint32_t va = ring0 + st * kRingUnit;
 #pragma unroll
             for (int s = 0; s < 8; ++s)
@@ -189,7 +186,8 @@ __device__ __forceinline__ void pr_issuer(const PrArgs &a, PrSmem &sm)
 // row's half; a row's two threads agree on the row's reference max (they
 // compute it from the same shared values).  In the epilogue the thread reads
 // O^T lane r (head dim r) for rows [64 hh, 64 hh + 64).
-__device__ __forceinline__ void pr_softmax(const PrArgs &a, PrSmem &sm, int warp, int lane)
+template <class A>
+__device__ __forceinline__ void pr_softmax(const A &a, PrSmem &sm, int warp, int lane)
 {
     const AttnParams &p = a.p;
     const int wq = warp & 3;
@@ -428,7 +426,7 @@ __device__ __forceinline__ void pr_softmax(const PrArgs &a, PrSmem &sm, int warp
 }
 
 template <bool kG>
-__global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_constant__ PrArgs a)
+__global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_constant__ PrArgs<kG> a)
 {
     extern __shared__ uint8_t smem_raw[];
     PrSmem &sm = *reinterpret_cast<PrSmem *>(
@@ -438,8 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
     const int lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NU; ++s) {
-            // a gathered unit completes with one arrival per producer lane
-            mbar_init(&sm.full[s], kG ? 32 : 1);
+            mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.q_full, 8);
@@ -468,15 +465,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_prompt_kernel(const __grid_c
 
     if (warp == 0) {
         if constexpr (kG) {
-            ring_producer_gather<1, NU>(a.p, sm, lane);
+            ring_producer_pieces<1, NU>(a.p, a.kmap, a.vmap, sm, lane);
         } else {
             if (lane == 0)
-                ring_producer<1, NU>(a.p, &a.kmap, &a.vmap, sm);
+                ring_producer<1, NU>(a.p, a.kmap, a.vmap, sm);
             __syncwarp();
         }
     } else if (warp == 1) {
         if (lane == 0)
-            pr_issuer<kG>(a, sm);
+            pr_issuer(a, sm);
         __syncwarp();
     } else {
         pr_softmax(a, sm, warp, lane);
@@ -503,28 +500,33 @@ bool prompt_supported(const AttnParams &p)
     return p.D == DD && pool_rows_fit(p);
 }
 
-cudaError_t launch_attn_prompt(const AttnParams &p, int grid, cudaStream_t stream)
+template <bool kG>
+cudaError_t launch_prompt(const AttnParams &p, int grid, cudaStream_t stream)
 {
-    PrArgs a;
+    PrArgs<kG> a;
     a.p = p;
-    if (!make_pool_map(&a.kmap, p.k_pool, p, PT) || !make_pool_map(&a.vmap, p.v_pool, p, PT))
-        return cudaErrorInvalidValue;
-    // pages that are a multiple of 128 positions hold whole tiles (TMA boxes);
-    // any other page size is gathered
-    if (p.P % PT != 0) {
-        static std::atomic<bool> configured[kMaxDevices];
-        const cudaError_t e = set_smem_limit_once(attn_prompt_kernel<true>, kPrSmemBytes, configured);
-        if (e != cudaSuccess)
-            return e;
-        return launch_dependent(attn_prompt_kernel<true>, dim3(grid), dim3(kThreads), kPrSmemBytes,
-                                stream, a);
+    // one box of a whole 128-position tile, or boxes of 1, 2, 4, ..., 128 rows
+    // for tiles assembled from page pieces
+    for (int h = 0; h < (kG ? kBoxHeights : 1); ++h) {
+        const int rows = kG ? 1 << h : PT;
+        if (!make_pool_map(&a.kmap[h], p.k_pool, p, rows) ||
+            !make_pool_map(&a.vmap[h], p.v_pool, p, rows))
+            return cudaErrorInvalidValue;
     }
     static std::atomic<bool> configured[kMaxDevices];
-    const cudaError_t e = set_smem_limit_once(attn_prompt_kernel<false>, kPrSmemBytes, configured);
+    const cudaError_t e = set_smem_limit_once(attn_prompt_kernel<kG>, kPrSmemBytes, configured);
     if (e != cudaSuccess)
         return e;
-    return launch_dependent(attn_prompt_kernel<false>, dim3(grid), dim3(kThreads), kPrSmemBytes,
+    return launch_dependent(attn_prompt_kernel<kG>, dim3(grid), dim3(kThreads), kPrSmemBytes,
                             stream, a);
+}
+
+// Pages that are a multiple of 128 positions hold whole tiles (one TMA box);
+// other page sizes assemble each tile from page pieces.
+cudaError_t launch_attn_prompt(const AttnParams &p, int grid, cudaStream_t stream)
+{
+    return p.P % PT != 0 ? launch_prompt<true>(p, grid, stream)
+                         : launch_prompt<false>(p, grid, stream);
 }
 
 }  // namespace tfp

@@ -193,23 +193,6 @@ __device__ __forceinline__ void bulk_wait_read()
 // Waits until all of the thread's bulk groups are complete (writes performed).
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// 16-byte asynchronous copy (cp.async, cached in L2 only) from global to
-// shared memory; both addresses 16-byte aligned.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint64_t policy)
-{
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)),
-                 "l"(src), "l"(policy)
-                 : "memory");
-}
-
-// One arrival on `bar`, made once every cp.async this thread issued so far has
-// completed; the arrival counts toward the barrier's expected count (noinc).
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
 // L2 policy for data read once per call (K/V streams): evict first.
 __device__ __forceinline__ uint64_t l2_evict_first_policy()
 {

@@ -119,83 +119,91 @@ __device__ __forceinline__ void ring_producer(const AttnParams &p, const CUtenso
     }
 }
 
-// ---- page sizes that are not a multiple of 128: tiles gathered row by row ----
+// ---- page sizes that are not a multiple of 128: tiles assembled from pages ----
 //
-// A 128-position tile may then straddle pages, and a TMA box cannot follow
-// the table.  The producer warp instead copies every position's row (128
-// dims of K or V: 256 bytes, 16 chunks of 16 bytes) with cp.async into the
-// same 128-byte-swizzled layout the TMA boxes produce, so the MMAs read the
-// ring unchanged.  Each lane arrives on the unit's full barrier once its own
-// copies have landed (32 arrivals per phase).  The consumers then issue a
-// proxy fence before the MMAs read the unit (cp.async writes through the
-// generic proxy).
+// A 128-position tile may then straddle pages, and one box of 128 rows cannot
+// follow the table.  The tile is cut into pieces, one per page it touches,
+// and each piece of n rows is loaded with one 2-D TMA box per set bit of n
+// (box heights 1, 2, 4, ..., 128 rows, one tensor map each), each landing at
+// its own tile row.  The 128-byte swizzle is a function of the shared-memory
+// address, so the pieces form the same layout a single 128-row box gives and
+// the MMAs read the ring unchanged.  Rows at or past the stream's end are not
+// loaded (their K rows are masked and their V rows zeroed before use), and
+// the unit completes on its full barrier by bytes.
 
-// Pool rows of the tile's positions: lane l holds position tpos + 32 i + l in
-// y[i]; -1 for a position at or past the stream's end (never read: its K row
-// is masked and its V row zeroed before use) or on a page outside the pool
-// (never read; flagged).  Table entries past the stream's end are not read.
-struct TileRows {
-    int y[4];
+constexpr int kBoxHeights = 8;  // tensor maps of boxes 1, 2, 4, ..., 128 rows high
+
+// The pages of a tile's valid rows [tpos, tpos + nvalid): the first is page
+// lp0, entered at slot off0; lane l holds the id of page lp0 + l (the first 32
+// pages the rows touch).  Table entries past the stream's pages are not read.
+struct TilePages {
+    int lp0, off0;
+    int id;
 };
 
-__device__ __forceinline__ TileRows tile_rows(const AttnParams &p, const int32_t *trow, int kh,
-                                              int tpos, int len, int lane)
+__device__ __forceinline__ TilePages tile_pages(const AttnParams &p, const int32_t *trow, int tpos,
+                                                int nvalid, int lane)
 {
-    TileRows t;
-    bool bad = false;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int pos = tpos + 32 * i + lane;
-        int y = -1;
-        if (pos < len) {
-            const int lp = pos / p.P;
-            const int page = __ldg(trow + lp);
-            if (page >= 0 && page < p.n_pages)
-                y = (page * p.Hkv + kh) * p.P + (pos - lp * p.P);
-            else
-                bad = true;
-        }
-        t.y[i] = y;
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0)
-        set_flag(p.flags, kDevBadPage);
+    TilePages t;
+    t.lp0 = tpos / p.P;
+    t.off0 = tpos - t.lp0 * p.P;
+    // page lp0 + lane starts at tile row lane * P - off0: does it hold a valid row?
+    const bool mine = (int64_t)lane * p.P < (int64_t)t.off0 + nvalid;
+    t.id = mine ? __ldg(trow + t.lp0 + lane) : 0;
     return t;
 }
 
-// The whole warp: waits until slot st is free, then copies dims [128 kb,
-// 128 kb + 128) of the tile's rows from `pool` into it.  False (uniform) when
-// the wait gave up.
+// The whole warp (lane 0 issues): waits until slot st is free, then loads
+// dims [128 kb, 128 kb + 128) of the tile's valid rows through `maps` (the K
+// or V pool, box heights 2^h) into it.  False (uniform) when the wait gave up.
 template <class Sm>
-__device__ __forceinline__ bool gather_unit(const AttnParams &p, Sm &sm, int st, uint32_t parity,
-                                            const __nv_bfloat16 *pool, const TileRows &rows,
-                                            int kb, int lane, uint64_t pol)
+__device__ __forceinline__ bool pieces_unit(const AttnParams &p, Sm &sm, int st, uint32_t parity,
+                                            const CUtensorMap *maps, const TilePages &tp,
+                                            const int32_t *trow, int kh, int nvalid, int kb,
+                                            int lane, uint64_t pol)
 {
     bool ok = true;
-    if (lane == 0)
+    if (lane == 0) {
         ok = pwait(sm, &sm.empty[st], parity, p.flags, kWaitEmpty);
+        if (ok)
+            mbar_arrive_expect_tx(&sm.full[st], (uint32_t)nvalid * 256u);
+    }
     if (!__shfl_sync(0xffffffffu, ok, 0))
         return false;
-    const int ch = lane & 15;  // the lane's 16-byte chunk of a row: dims [8 ch, 8 ch + 8)
-    uint8_t *const dst = sm.ring[st] + (ch >> 3) * kRingBox;
-    const __nv_bfloat16 *const src = pool + kb * 128 + ch * 8;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            // rows 32 i + 2 k (lanes 0-15) and 32 i + 2 k + 1 (lanes 16-31)
-            const int j = 2 * k + (lane >> 4);
-            const int y = __shfl_sync(0xffffffffu, rows.y[i], j);
-            if (y >= 0)
-                cp_async16(dst + sw128_off(32 * i + j, ch & 7), src + (size_t)y * p.D, pol);
+    // one piece per page: rows [r, r + n) of the tile from page lp0 + j,
+    // slots [off, off + n)
+    int off = tp.off0;
+    for (int r = 0, j = 0; r < nvalid; ++j) {
+        const int n = min(nvalid - r, p.P - off);
+        int page = j < 32 ? __shfl_sync(0xffffffffu, tp.id, j) : __ldg(trow + tp.lp0 + j);
+        if (lane == 0) {
+            if (page < 0 || page >= p.n_pages) {
+                // never read: page 0 stands in (the stream's outputs are flagged)
+                set_flag(p.flags, kDevBadPage);
+                page = 0;
+            }
+            int row = r, y = (page * p.Hkv + kh) * p.P + off;
+            for (int m = n; m != 0;) {
+                const int h = 31 - __clz(m);  // the largest box that fits: 2^h rows
+                tma_load_2d(sm.ring[st] + row * 128, &maps[h], 128 * kb, y, &sm.full[st], pol);
+                tma_load_2d(sm.ring[st] + kRingBox + row * 128, &maps[h], 128 * kb + 64, y,
+                            &sm.full[st], pol);
+                row += 1 << h;
+                y += 1 << h;
+                m -= 1 << h;
+            }
         }
+        r += n;
+        off = 0;
     }
-    cp_async_arrive(&sm.full[st]);
     return true;
 }
 
-// The whole producer warp: the unit order of ring_producer, gathered.
+// The whole producer warp: the unit order of ring_producer, assembled from
+// pieces.  kmaps / vmaps: kBoxHeights tensor maps each.
 template <int DB, int NU, class Sm>
-__device__ __forceinline__ void ring_producer_gather(const AttnParams &p, Sm &sm, int lane)
+__device__ __forceinline__ void ring_producer_pieces(const AttnParams &p, const CUtensorMap *kmaps,
+                                                     const CUtensorMap *vmaps, Sm &sm, int lane)
 {
     const uint64_t pol = l2_evict_first_policy();
     SegCursor cur;
@@ -203,33 +211,38 @@ __device__ __forceinline__ void ring_producer_gather(const AttnParams &p, Sm &sm
     WorkItem it;
     uint32_t U = 0;  // units issued
     bool ok = true;
-    auto put_tile = [&](const __nv_bfloat16 *pool, const TileRows &rows) {
+    auto put_tile = [&](const CUtensorMap *maps, const TilePages &tp, const int32_t *trow, int kh,
+                        int nvalid) {
 #pragma unroll 1
         for (int kb = 0; ok && kb < DB; ++kb) {
-            ok = gather_unit(p, sm, (int)(U % NU), ((U / NU) & 1u) ^ 1u, pool, rows, kb, lane, pol);
+            ok = pieces_unit(p, sm, (int)(U % NU), ((U / NU) & 1u) ^ 1u, maps, tp, trow, kh, nvalid,
+                             kb, lane, pol);
             U += ok ? 1u : 0u;
         }
     };
+    constexpr int PT = kRingTile;
     while (ok && cur.next(p, it)) {
-        const int n = (it.key1 - it.key0 + kRingTile - 1) / kRingTile;
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
-        TileRows r0 = tile_rows(p, trow, it.kh, it.key0, it.len, lane);
-        put_tile(p.k_pool, r0);
+        // rows and page ids of tiles t, t + 1 and t + 2 (the page ids are read
+        // two tiles before their first use)
+        auto nvalid = [&](int t) { return min(PT, it.len - (it.key0 + t * PT)); };
+        TilePages t0 = tile_pages(p, trow, it.key0, nvalid(0), lane);
+        TilePages t1 = n > 1 ? tile_pages(p, trow, it.key0 + PT, nvalid(1), lane) : t0;
+        put_tile(kmaps, t0, trow, it.kh, nvalid(0));
         for (int t = 0; ok && t < n; ++t) {
-            const int pos = it.key0 + t * kRingTile;
-            TileRows r1 = r0;
-            if (t + 1 < n) {
-                r1 = tile_rows(p, trow, it.kh, pos + kRingTile, it.len, lane);
-                put_tile(p.k_pool, r1);
-            }
+            const int pos = it.key0 + t * PT;
+            const TilePages t2 = t + 2 < n ? tile_pages(p, trow, pos + 2 * PT, nvalid(t + 2), lane) : t1;
+            if (t + 1 < n)
+                put_tile(kmaps, t1, trow, it.kh, nvalid(t + 1));
             if (ok)
-                put_tile(p.v_pool, r0);
-            r0 = r1;
+                put_tile(vmaps, t0, trow, it.kh, nvalid(t));
+            t0 = t1;
+            t1 = t2;
         }
     }
     if (lane == 0) {
-        // Let the copies in flight land before the CTA can exit (a unit's
-        // phase completes once every lane's copies of it have landed).
+        // let the copies in flight land before the CTA can exit
         const uint32_t nf = U < (uint32_t)NU ? U : (uint32_t)NU;
         for (uint32_t k = 1; k <= nf; ++k) {
             const uint32_t v = U - k;

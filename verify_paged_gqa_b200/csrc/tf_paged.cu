@@ -132,9 +132,20 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     // too (decode at GQA 4): its two MMA issuers keep pace with HBM at any
     // clock, where the CUDA-core kernel's FMAs fall behind under the power
     // cap (12 x 40,960 decode: 341 -> 296 us per call).  Head dim 512 keeps
-    // such calls on the CUDA-core kernel.  Any page size runs on the
-    // tensor-core kernels (tiles that straddle pages are gathered row by
-    // row); only pools past 2^31 rows fall back to the CUDA-core kernel.
+    // such calls on the CUDA-core kernel.  Pages that are not a multiple of
+    // 128 positions: the tensor-core kernels assemble each tile from page
+    // pieces, one TMA box per set bit of a piece's length, so small pages
+    // cost many box loads per tile.  For a single 4-row block (decode at
+    // GQA <= 4) the CUDA-core kernel, which copies pieces into its own
+    // smaller tiles, is then faster below 128 positions unless the page is a
+    // multiple of 64 (12 x 40,960 decode, GB/s, CUDA-core / tensor-core:
+    // pages of 37 3,378 / 1,915; 48 3,995 / 3,175; 64 5,045 / 5,190; 96
+    // 5,368 / 4,830; 100 4,208 / 3,599; 200 4,555 / 4,951; 509 4,697 /
+    // 5,527).  Several row blocks would each re-read the K/V on the CUDA-core
+    // kernel, so larger blocks always take the tensor cores (verify
+    // 4 x 131,072 in pages of 64: 311 against 4,467 GB/s).  Pools past 2^31
+    // rows run on the CUDA-core kernel.
+    const bool small_odd_pages = p.P < 128 && p.P % 64 != 0;
     plan->kernel = Kernel::kSimt;
     p.RB = kSimtRows;
     if (tree) {
@@ -154,7 +165,7 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
             return TF_EUNSUPPORTED;
         plan->kernel = Kernel::kPm;
         p.RB = nr;
-    } else if (M > kSimtRows || p.D == 128) {
+    } else if (M > kSimtRows || (p.D == 128 && !small_odd_pages)) {
         const int nr = pm_rows(p);
         if (nr > 0) {
             plan->kernel = Kernel::kPm;
