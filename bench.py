@@ -737,7 +737,7 @@ def main():
         # head dim 256), each timed the same way
         line["variants"] = []
         for name in ("gqa12_verify", "gqa16_hd512_decode", "hd256_verify", "tree_verify_4x131k",
-                     "decode_12x40k_p37"):
+                     "decode_12x40k_p37", "decode_64x2k"):
             line["variants"].append(measure_other(name, args, barrier, dist, world, local))
             torch.cuda.empty_cache()
         line["state_copy"] = measure_state_copy(args, barrier, dist, world, local)

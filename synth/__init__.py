@@ -151,6 +151,11 @@ WORKLOADS = {
     # the decode workload in pages of 37 positions (tiles straddle pages)
     "decode_12x40k_p37": Workload("decode_12x40k_p37", 12, 8, 4, 128, 37, 1, seed=12,
                                   lens=(40960,) * 12),
+    # many short streams (a serving batch early in its contexts): 64 x 2,048
+    # and 256 x 512 positions, the decode workload's heads
+    "decode_64x2k": Workload("decode_64x2k", 64, 8, 4, 128, 512, 1, seed=14, lens=(2048,) * 64),
+    "decode_256x512": Workload("decode_256x512", 256, 8, 4, 128, 512, 1, seed=15,
+                               lens=(512,) * 256),
     # smaller copies of the decode and verify workloads for profiler captures
     # (still larger than the 126 MB L2)
     "decode_12x8k": Workload("decode_12x8k", 12, 8, 4, 128, 512, 1, seed=6, lens=(8192,) * 12),

@@ -98,12 +98,14 @@ def test_nan_never_reaches_output_and_negative_control_goes_red():
 
 
 @pytest.mark.parametrize("d,G,P,W,lens,tree", [
-    (128, 4, 512, 1, [1300, 600, 2049], False),     # decode, position-major kernel
+    (128, 4, 512, 1, [1300, 600, 2049], False),     # decode, short contexts: CUDA-core kernel
+    (128, 4, 512, 1, [7000, 600, 2049], False),     # decode, position-major kernel
     (128, 8, 512, 8, [1300, 600, 2049], False),     # verify, position-major kernel
     (512, 4, 512, 1, [1300, 600, 2049], False),     # head dim 512 decode, CUDA-core kernel
     (256, 8, 512, 4, [1300, 600, 2049], False),     # head dim 256 verify
     (128, 4, 512, 100, [1300, 600, 2049], False),   # prompt chunk, row-major kernel
-    (128, 4, 37, 4, [1300, 600, 2049], False),      # pages of 37, CUDA-core kernel
+    (128, 4, 37, 4, [1300, 600, 2049], False),      # pages of 37, tiles from page pieces
+    (128, 4, 37, 1, [1300, 600, 2049], False),      # pages of 37, CUDA-core decode
     (128, 8, 512, 5, [1300, 600, 2049], True),      # tree masks
 ])
 def test_fill_of_unused_slots_changes_no_output_bit(d, G, P, W, lens, tree):

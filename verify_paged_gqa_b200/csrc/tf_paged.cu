@@ -83,6 +83,10 @@ constexpr int kEntryPm128 = 6;
 constexpr int kEntryPrompt = 8;
 constexpr int kEntrySimt = 0;
 
+// Decode blocks at head dim 128 take the position-major kernel from this
+// max_len on (measured crossover near 5,700 positions).
+constexpr int kPmDecodeMinLen = 6144;
+
 struct Plan {
     AttnParams p;
     int grid;
@@ -146,6 +150,14 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
     // 4 x 131,072 in pages of 64: 311 against 4,467 GB/s).  Pools past 2^31
     // rows run on the CUDA-core kernel.
     const bool small_odd_pages = p.P < 128 && p.P % 64 != 0;
+    // A decode block also stays on the CUDA-core kernel for short contexts:
+    // the position-major kernel pays about six tiles (768 positions) to start
+    // each (stream, KV head) unit, which outweighs its steady-state lead
+    // below about 6,000 positions (GB/s, position-major / CUDA-core: 64 x
+    // 2,048 4,507 / 5,112; 256 x 512 3,207 / 3,638; 12 x 8,192 5,315 /
+    // 5,187; 12 x 40,960 6,875 / 6,061).  max_len bounds every stream, so the
+    // choice depends on host arguments only.
+    const bool long_context = st->max_len >= kPmDecodeMinLen;
     plan->kernel = Kernel::kSimt;
     p.RB = kSimtRows;
     if (tree) {
@@ -165,7 +177,7 @@ int make_plan(const tf_kv_pool *pool, const tf_streams *st, int32_t Hq, int32_t 
             return TF_EUNSUPPORTED;
         plan->kernel = Kernel::kPm;
         p.RB = nr;
-    } else if (M > kSimtRows || (p.D == 128 && !small_odd_pages)) {
+    } else if (M > kSimtRows || (p.D == 128 && !small_odd_pages && long_context)) {
         const int nr = pm_rows(p);
         if (nr > 0) {
             plan->kernel = Kernel::kPm;
