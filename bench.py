@@ -14,9 +14,11 @@ shuffled pool 1.2x the pages needed (TensorFold #1620's ``--parallel 12
 
 value  = algorithmic K/V bytes per step (visible positions x KV heads x
          head_dim x 2 bytes x {K, V}) / device time per step, whole job.
-e2e    = the same metric through the public API with host buffers: the
-         step's query and new rows copied from pinned host memory, the
-         output copied back, inside the timed region.
+e2e    = the same metric through the public API with host buffers: every
+         step's query and new rows copied from pinned host memory and its
+         output copied back, inside the timed region, on copy streams that
+         overlap the neighbouring steps' kernels (two sets of device
+         buffers, as a serving loop runs).
 roofline = the attention call (partial + merge kernels) alone, its K/V bytes
          over its CUDA-event time, against the measured HBM copy bandwidth.
 cpu_baseline = the fp64 CPU oracle timed on the host on a bounded sample.
@@ -362,29 +364,31 @@ class Workload:
                 kp, vp, tb, ln, q, self.tree, sc, out, ws, ml)
         torch.cuda.synchronize()
 
-    def parts(self, k_new=None, v_new=None, q=None):
-        """The step's (row write, attention) pairs, optionally on other input buffers."""
+    def parts(self, k_new=None, v_new=None, q=None, out=None):
+        """The step's (row write, attention) pairs, optionally on other input and
+        output buffers."""
         k_new = self.k_new if k_new is None else k_new
         v_new = self.v_new if v_new is None else v_new
         q = self.q if q is None else q
+        out = self.out if out is None else out
         tf, w = self.tf, self.w
         if self.chunk_lens is None:
             return [(lambda: tf.tf_kv_put_rows(self.k_pool, self.v_pool, self.table, self.lens,
                                                k_new, v_new, max_len=self.max_len),
                      lambda: self.attn_fn(self.k_pool, self.v_pool, self.table, self.lens, q,
-                                          w.scale, self.out, self.ws, self.max_len))]
+                                          w.scale, out, self.ws, self.max_len))]
         W = w.rows
-        out = []
+        pairs = []
         for c, lens_c in enumerate(self.chunk_lens):
             sl = slice(c * W, (c + 1) * W)
-            out.append((
+            pairs.append((
                 lambda sl=sl, lens_c=lens_c: tf.tf_kv_put_rows(
                     self.k_pool, self.v_pool, self.table, lens_c, k_new[:, sl], v_new[:, sl],
                     max_len=self.max_len),
                 lambda sl=sl, lens_c=lens_c: self.attn_fn(
                     self.k_pool, self.v_pool, self.table, lens_c, q[:, sl], w.scale,
-                    self.out[:, sl], self.ws, self.max_len)))
-        return out
+                    out[:, sl], self.ws, self.max_len)))
+        return pairs
 
     def step(self):
         for put, att in self.parts():
@@ -469,40 +473,71 @@ def time_steps(wl, steps, warmup, barrier, sampler=None, blocks=10):
 
 
 def time_e2e(wl, steps, warmup, barrier):
-    """Same steps through the public API from pinned host buffers (copies inside)."""
+    """The same steps through the public API from pinned host buffers, run as a
+    serving loop runs them: every step copies its query and new rows in from
+    pinned host memory and its output back, but on copy streams of their own
+    and into two sets of device buffers, so step k + 1's inputs cross PCIe
+    while step k computes, and step k's output crosses back while step k + 1
+    computes.  Every copy of every step lies inside the timed region (events
+    on the compute stream bracket all three streams)."""
     torch = wl.torch
     q_h = wl.q.cpu().pin_memory()
     k_h = wl.k_new.cpu().pin_memory()
     v_h = wl.v_new.cpu().pin_memory()
-    out_h = torch.empty(wl.out.shape, dtype=torch.float32).pin_memory()
-    q_d, k_d, v_d = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
-    parts = wl.parts(k_d, v_d, q_d)
+    out_h = [torch.empty(wl.out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    bufs = [(torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new),
+             torch.empty_like(wl.out)) for _ in range(2)]
+    parts = [wl.parts(k_d, v_d, q_d, out=o_d) for q_d, k_d, v_d, o_d in bufs]
+    comp = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready = [ev(), ev()]    # set b's inputs landed
+    computed = [ev(), ev()]    # the step on set b computed (its inputs are free again)
+    out_back = [ev(), ev()]    # set b's output copied back (its output buffer is free again)
 
-    def one():
-        q_d.copy_(q_h, non_blocking=True)
-        k_d.copy_(k_h, non_blocking=True)
-        v_d.copy_(v_h, non_blocking=True)
-        for put, att in parts:
+    def one(k):
+        b = k & 1
+        q_d, k_d, v_d, o_d = bufs[b]
+        with torch.cuda.stream(h2d_s):
+            if k >= 2:
+                h2d_s.wait_event(computed[b])
+            q_d.copy_(q_h, non_blocking=True)
+            k_d.copy_(k_h, non_blocking=True)
+            v_d.copy_(v_h, non_blocking=True)
+            in_ready[b].record(h2d_s)
+        comp.wait_event(in_ready[b])
+        if k >= 2:
+            comp.wait_event(out_back[b])
+        for put, att in parts[b]:
             put()
             att()
-        out_h.copy_(wl.out, non_blocking=True)
+        computed[b].record(comp)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(computed[b])
+            out_h[b].copy_(o_d, non_blocking=True)
+            out_back[b].record(d2h_s)
 
-    for _ in range(warmup):
-        one()
+    def run(n):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(comp)
+        h2d_s.wait_event(start)
+        d2h_s.wait_event(start)
+        for k in range(n):
+            one(k)
+        comp.wait_event(out_back[(n - 1) & 1])
+        end.record(comp)
+        return start, end
+
+    run(warmup)
     torch.cuda.synchronize()
     barrier()
-    stream = torch.cuda.current_stream()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(steps):
-        one()
-    end.record(stream)
+    start, end = run(steps)
     torch.cuda.synchronize()
     barrier()
     h2d = (q_h.numel() * q_h.element_size() + k_h.numel() * k_h.element_size()
            + v_h.numel() * v_h.element_size())
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size()
     return start.elapsed_time(end), h2d, d2h
 
 

@@ -89,12 +89,13 @@ extern "C" {
 #define TF_DEV_TIMEOUT 4u   /* a pipeline wait gave up (an internal error) */
 
 /* The pool: K and V pages, device memory, 16-byte aligned.
- * page_size may be any positive size (TensorFold #1620, Checks, the kernel-
- * contract bullet: the paged prompt kernel is checked over pages of 512, 37
- * and 64); head_dim must be 128, 256 or 512.  The tensor-core kernels need
- * page_size a multiple of 128: other sizes run on the CUDA-core kernel,
- * whose tiles may then straddle pages, and head dim 256 calls are refused
- * for them (TF_EUNSUPPORTED). */
+ * page_size may be any positive size at every head dim (TensorFold #1620,
+ * Checks, the kernel-contract bullet: the paged prompt kernel is checked
+ * over pages of 512, 37 and 64); head_dim must be 128, 256 or 512.  Pages
+ * that are not a multiple of 128 positions are read by tiles assembled from
+ * page pieces; the results do not depend on the page size.  Head dim 256
+ * calls are refused (TF_EUNSUPPORTED) for pools of more than 2^31 - 1 rows
+ * (n_pages * n_kv_heads * page_size). */
 typedef struct tf_kv_pool {
     void *k_pool;
     void *v_pool;
@@ -196,9 +197,7 @@ TF_API int tf_paged_attn_verify(const tf_kv_pool *pool, const tf_streams *stream
  *              (no context before the window and an empty mask) gets NaN.
  * Everything else (arguments, layouts, results, the workspace, errors) is
  * as tf_paged_attn_verify; TF_EINVAL also when tree_masks is null (with
- * n_streams > 0), and
- * TF_EUNSUPPORTED for head dim 256 with a page_size that is not a multiple
- * of 128.  Head dim 128
+ * n_streams > 0).  Head dim 128
  * calls with more than 64 query rows per KV head (G * rows) read each K/V
  * tile once per 64 rows. */
 TF_API int tf_paged_attn_verify_tree(const tf_kv_pool *pool, const tf_streams *streams,

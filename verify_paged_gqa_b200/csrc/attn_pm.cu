@@ -550,90 +550,97 @@ __device__ __forceinline__ void pm_softmax(const A &a, PmSmem<D, NR> &sm, int wa
     const int sw = tid & 7;
     const int R0 = 32 * h;               // first row of this thread
 
-    SegCursor cur;
-    cur.init(p, sm.range);
-    WorkItem it, nx;
-    uint32_t j = 0, u0 = 0;
     bool ok = true;
-    for (; cur.next(p, it); ++j) {
-        const int n = (it.key1 - it.key0 + PT - 1) / PT;
-        // --- the block's query rows into the Q tile; output offsets ---------
+    // The query rows of segment jj (unit w) into the Q tile, the rows' output
+    // offsets, and under tree masks the rows' window masks; then the issuer
+    // may run the segment's QK.  `after` is the cursor past segment jj.
+    auto load_q = [&](const WorkItem &w, uint32_t jj, const SegCursor &after) {
+        constexpr int kPer = NR * D / 8 / NT;  // 16-byte chunks per thread
+        static_assert(kPer % 4 == 0, "Q chunks");
+        if (st < NR) {
+            const int m = w.b * NR + st;
+            long long off = -1;
+            if (m < p.M) {
+                const int wr = m / p.G;
+                const int hq = w.kh * p.G + (m - wr * p.G);
+                off = (((long long)w.s * p.W + wr) * p.Hq + hq) * D;
+            }
+            sm.rowoff[jj & 1u][st] = off;
+        }
         {
-            constexpr int kPer = NR * D / 8 / NT;  // 16-byte chunks per thread
-            static_assert(kPer % 4 == 0, "Q chunks");
-            if (st < NR) {
-                const int m = it.b * NR + st;
-                long long off = -1;
+            uint4 qv[kPer];
+#pragma unroll
+            for (int c = 0; c < kPer; ++c) {
+                const int f = st + NT * c;
+                const int r = f / (D / 8), k = f % (D / 8);
+                const int m = w.b * NR + r;
+                qv[c] = make_uint4(0, 0, 0, 0);
                 if (m < p.M) {
                     const int wr = m / p.G;
-                    const int hq = it.kh * p.G + (m - wr * p.G);
-                    off = (((long long)it.s * p.W + wr) * p.Hq + hq) * D;
+                    const int hq = w.kh * p.G + (m - wr * p.G);
+                    qv[c] = __ldg(reinterpret_cast<const uint4 *>(
+                                      p.q + (((size_t)w.s * p.W + wr) * p.Hq + hq) * D) +
+                                  k);
                 }
-                sm.rowoff[j & 1u][st] = off;
             }
-            // (already complete in practice: the previous segment's last PV,
-            // waited for below, was issued after its last QK)
-            ok = pwait(sm, &sm.q_free, (j & 1u) ^ 1u, p.flags, kWaitQEmpty) && ok;
-            {
-                uint4 qv[kPer];
+            // the Q tile is free once the previous segment's last QK completed
+            ok = pwait(sm, &sm.q_free, (jj & 1u) ^ 1u, p.flags, kWaitQEmpty) && ok;
 #pragma unroll
-                for (int c = 0; c < kPer; ++c) {
-                    const int f = st + NT * c;
-                    const int r = f / (D / 8), k = f % (D / 8);
-                    const int m = it.b * NR + r;
-                    qv[c] = make_uint4(0, 0, 0, 0);
-                    if (m < p.M) {
-                        const int wr = m / p.G;
-                        const int hq = it.kh * p.G + (m - wr * p.G);
-                        qv[c] = __ldg(reinterpret_cast<const uint4 *>(
-                                          p.q + (((size_t)it.s * p.W + wr) * p.Hq + hq) * D) +
-                                      k);
-                    }
-                }
-#pragma unroll
-                for (int c = 0; c < kPer; ++c) {
-                    const int f = st + NT * c;
-                    const int r = f / (D / 8), k = f % (D / 8);
-                    *reinterpret_cast<uint4 *>(sm.q + (k >> 3) * (NR * 128) + sw128_off(r, k & 7)) =
-                        qv[c];
-                }
+            for (int c = 0; c < kPer; ++c) {
+                const int f = st + NT * c;
+                const int r = f / (D / 8), k = f % (D / 8);
+                *reinterpret_cast<uint4 *>(sm.q + (k >> 3) * (NR * 128) + sw128_off(r, k & 7)) =
+                    qv[c];
             }
-            // the next segment's query rows into L2 (128-byte lines)
-            SegCursor ahead = cur;
-            if (ahead.next(p, nx)) {
-                constexpr int kLines = NR * D * 2 / 128;
-                for (int f = st; f < kLines; f += NT) {
-                    const int r = f / (D / 64), k = f % (D / 64);
-                    const int m = nx.b * NR + r;
-                    if (m < p.M) {
-                        const int wr = m / p.G;
-                        const int hq = nx.kh * p.G + (m - wr * p.G);
-                        const __nv_bfloat16 *src =
-                            p.q + (((size_t)nx.s * p.W + wr) * p.Hq + hq) * D + k * 64;
-                        asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
-                    }
-                }
-            }
-            if (kTree && st < NR / 32 * 8) {
-                // the block's rows that see window row c, from the stream's masks
-                const int hh = st >> 3, c = st & 7;
-                uint32_t wv = 0;
-                if (c < p.W) {
-                    const uint8_t *tm = p.tree + (size_t)it.s * p.W;
-                    for (int r = 0; r < 32; ++r) {
-                        const int m = it.b * NR + 32 * hh + r;
-                        if (m < p.M && ((__ldg(tm + m / p.G) >> c) & 1))
-                            wv |= 1u << r;
-                    }
-                }
-                sm.rowvis[hh][c] = wv;
-            }
-            fence_async_smem();
-            named_barrier(1, NT);
-            if (st == 0)
-                mbar_arrive(&sm.q_full);
         }
+        // the following segment's query rows into L2 (128-byte lines)
+        SegCursor ahead = after;
+        WorkItem nx2;
+        if (ahead.next(p, nx2)) {
+            constexpr int kLines = NR * D * 2 / 128;
+            for (int f = st; f < kLines; f += NT) {
+                const int r = f / (D / 64), k = f % (D / 64);
+                const int m = nx2.b * NR + r;
+                if (m < p.M) {
+                    const int wr = m / p.G;
+                    const int hq = nx2.kh * p.G + (m - wr * p.G);
+                    const __nv_bfloat16 *src =
+                        p.q + (((size_t)nx2.s * p.W + wr) * p.Hq + hq) * D + k * 64;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
+                }
+            }
+        }
+        if (kTree && st < NR / 32 * 8) {
+            // the block's rows that see window row c, from the stream's masks
+            // (every thread read the previous segment's masks before its last
+            // tile's vote)
+            const int hh = st >> 3, c = st & 7;
+            uint32_t wv = 0;
+            if (c < p.W) {
+                const uint8_t *tm = p.tree + (size_t)w.s * p.W;
+                for (int r = 0; r < 32; ++r) {
+                    const int m = w.b * NR + 32 * hh + r;
+                    if (m < p.M && ((__ldg(tm + m / p.G) >> c) & 1))
+                        wv |= 1u << r;
+                }
+            }
+            sm.rowvis[hh][c] = wv;
+        }
+        fence_async_smem();
+        named_barrier(1, NT);
+        if (st == 0)
+            mbar_arrive(&sm.q_full);
+    };
 
+    SegCursor cur;
+    cur.init(p, sm.range);
+    WorkItem it;
+    uint32_t j = 0, u0 = 0;
+    bool have = cur.next(p, it);
+    if (have)
+        load_q(it, 0, cur);
+    for (; have; ++j) {
+        const int n = (it.key1 - it.key0 + PT - 1) / PT;
         float l[32];
 #pragma unroll
         for (int r = 0; r < 32; ++r)
@@ -677,9 +684,7 @@ __device__ __forceinline__ void pm_softmax(const A &a, PmSmem<D, NR> &sm, int wa
                     for (int r = 0; r < 32; ++r)
                         x[r] = pm_sees<kTree>(r, rvis, vis) ? x[r] : NEG_INF;
                 }
-#pragma unroll
-                for (int r = 0; r < 32; ++r)
-                    mx = fmaxf(mx, x[r]);
+                mx = max_tree(x);
                 slow = block_any<NT>(mx > kRescaleLog2);
             }
             if (slow) {
@@ -813,6 +818,16 @@ __device__ __forceinline__ void pm_softmax(const A &a, PmSmem<D, NR> &sm, int wa
                 mbar_arrive(&sm.p_full[u & 1u]);
         }
 
+        // --- the next segment's query rows, so that the issuer runs its first QK
+        // while this segment's rows are written (the Q tile is free once this
+        // segment's last QK completed; the next segment's first PV, which
+        // overwrites O^T, waits for its P, written after this epilogue) ----------
+        WorkItem nx;
+        SegCursor ahead = cur;
+        const bool have_nx = ahead.next(p, nx);
+        if (have_nx)
+            load_q(nx, j + 1, ahead);
+
         // --- the segment's last PV, then the rows' results ------------------------
         const uint32_t ulast = u0 + n - 1;
         ok = pwait(sm, &sm.o_done[ulast & 1u], (ulast >> 1) & 1u, p.flags, kWaitEmpty) && ok;
@@ -857,6 +872,9 @@ __device__ __forceinline__ void pm_softmax(const A &a, PmSmem<D, NR> &sm, int wa
         }
         tc_fence_before();
         u0 += n;
+        cur = ahead;
+        it = nx;
+        have = have_nx;
     }
 }
 

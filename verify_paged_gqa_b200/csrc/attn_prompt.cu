@@ -287,10 +287,7 @@ __device__ __forceinline__ void pr_softmax(const A &a, PrSmem &sm, int warp, int
                 for (int k = 0; k < 64; ++k)
                     s[k] = k < vis ? s[k] : NEG_INF;
             }
-            float hmax = NEG_INF;
-#pragma unroll
-            for (int k = 0; k < 64; ++k)
-                hmax = fmaxf(hmax, s[k]);
+            const float hmax = max_tree(s);
             const float hm = hmax == NEG_INF ? NEG_INF : hmax * sl;
             // a half that would move the row's reference calls for the slow path
             const bool hgrow = hm != NEG_INF && (mref == NEG_INF || hm > mref + kRescaleLog2);

@@ -201,6 +201,27 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy()
     return pol;
 }
 
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Maximum of v[0 .. N) (N >= 4, N even) in four independent chains of
+// three-input maxima: N / 2 instructions, a dependency depth of about N / 8.
+template <int N>
+__device__ __forceinline__ float max_tree(const float (&v)[N])
+{
+    static_assert(N >= 4 && N % 2 == 0, "max_tree");
+    float c[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+    for (int k = 4; k < N; k += 2)
+        c[(k / 2) & 3] = fmax3(c[(k / 2) & 3], v[k], v[k + 1]);
+    return fmaxf(fmax3(c[0], c[1], c[2]), c[3]);
+}
+
 __device__ __forceinline__ float fast_exp2(float x)
 {
     float y;
