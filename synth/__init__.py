@@ -162,6 +162,9 @@ WORKLOADS = {
     "decode_12x8k_p37": Workload("decode_12x8k_p37", 12, 8, 4, 128, 37, 1, seed=13,
                                  lens=(8192,) * 12),
     "verify_4x16k": Workload("verify_4x16k", 4, 4, 8, 128, 512, 8, seed=7, lens=(16384,) * 4),
+    # the verify copy in pages of 64 (tensor-core tiles assembled from page pieces)
+    "verify_4x16k_p64": Workload("verify_4x16k_p64", 4, 4, 8, 128, 64, 8, seed=16,
+                                 lens=(16384,) * 4),
 }
 
 
