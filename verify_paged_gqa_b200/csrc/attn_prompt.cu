@@ -4,10 +4,9 @@
 //
 // TensorFold #1620 ("Kolibri-1's full layers take their K/V from pages of
 // the core pool"), opening comment, "Reads": prompt rows attend over keys
-// read through the page table, causally.  Such a block is tensor bound, and
-// one tcgen05.mma (K = 16) costs about 120 cycles to issue for any N up to
-// 128 and 160 cycles at N = 256, so the kernel is built to issue few, wide
-// instructions per 128-position tile:
+// read through the page table, causally.  Such a block is tensor bound.  Per
+// 128-position tile the kernel issues 16 MMAs, which the tensor pipe runs at
+// its peak rate in 1,536 cycles (N / 2 cycles per K = 16 step at M = 128):
 //
 //   S    = Q K^T                  M = 128 rows, N = 128 positions, 8 MMAs,
 //                                 Q in tensor memory
