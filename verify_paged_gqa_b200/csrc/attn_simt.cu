@@ -16,9 +16,11 @@
 //                 double-buffered shared slot and streams K and V tiles of TK
 //                 positions into a ring of NSTAGE stages with bulk copies
 //                 (TMA engine, no tensor map: a tile of one page and KV head
-//                 is one contiguous run; with a page size that is not a
-//                 multiple of TK a tile may straddle pages and takes one copy
-//                 per page piece).  Page ids are read one page early.
+//                 is one contiguous run).  With a page size that is not a
+//                 multiple of TK a tile may straddle pages: tiles are then
+//                 armed four at a time (a quad of contiguous stages, complete
+//                 on one barrier) and one copy covers a page's run across
+//                 them.  Page ids are read one page early.
 //   other warps   consumers: tile T of the CTA's sequence goes to consumer
 //                 warp T % NCW.  A warp keeps its own online-softmax state
 //                 (running max m, running sum l, unnormalised O) for the four
@@ -81,7 +83,10 @@ struct SimtSmem {
     static constexpr int NSTAGE = SimtCfg<D>::NSTAGE;
     static constexpr int NCW = SimtCfg<D>::NCW;
     static constexpr int TILE_BYTES = TK * D * 2;
-    alignas(128) uint8_t kv[NSTAGE][2][TILE_BYTES];
+    // K and V rings: consecutive stages are contiguous, so a copy of a page
+    // piece may run across the stages of one quad (below)
+    alignas(128) uint8_t kring[NSTAGE][TILE_BYTES];
+    alignas(128) uint8_t vring[NSTAGE][TILE_BYTES];
     alignas(16) __nv_bfloat16 qbuf[2][kR][D];      // the segment's query rows (double buffer)
     alignas(16) float pbuf[NCW][TK][2 * kR];        // per key: p0,p0,p1,p1,p2,p2,p3,p3
     alignas(16) float wo[NCW][kR][D];               // parked warp states
@@ -180,6 +185,15 @@ __device__ __forceinline__ bool wait_tag(SimtSmem<D> &sm, int stage, uint32_t T,
     return true;
 }
 
+// Adds `bytes` to the transaction count of the barrier's current phase (no
+// arrival).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 // Copies the four query rows of segment `it` into q slot (j & 1).
 template <int D>
 __device__ __forceinline__ bool producer_q(const AttnParams &p, SimtSmem<D> &sm,
@@ -218,42 +232,80 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
     if (have && producer_q<D>(p, sm, it, 0, pol))
         q_issued = 1;
     int32_t page_next = have ? __ldg(p.table + (int64_t)it.s * p.table_stride + it.key0 / p.P) : 0;
+    // tiles assembled from page pieces: the quad being armed and the pending
+    // copy (pc_n positions of page pc_page, KV head pc_kh, from offset pc_off,
+    // into ring rows from pc_row)
+    const bool quads = p.P % TK != 0;
+    static_assert(NSTAGE % 4 == 0, "quads of stages");
+    int quad = -1;
+    int pc_n = 0, pc_pos = 0, pc_row = 0, pc_kh = 0, pc_off = 0;
+    int32_t pc_page = 0;
+    auto flush = [&]() {
+        if (pc_n == 0)
+            return;
+        uint64_t *bar = &sm.full[(quad * 4 + 3) % NSTAGE];
+        const uint32_t nb = static_cast<uint32_t>(pc_n) * D * 2u;
+        if (pc_page >= 0 && pc_page < p.n_pages) {
+            const size_t off = (((size_t)pc_page * p.Hkv + pc_kh) * p.P + pc_off) * D;
+            mbar_expect_tx(bar, 2u * nb);
+            bulk_g2s(&sm.kring[0][0] + (size_t)pc_row * D * 2, p.k_pool + off, nb, bar, pol);
+            bulk_g2s(&sm.vring[0][0] + (size_t)pc_row * D * 2, p.v_pool + off, nb, bar, pol);
+        } else {
+            set_flag(p.flags, kDevBadPage);
+        }
+        pc_n = 0;
+    };
     while (have && !sm.abort_flag) {
         SegCursor ahead = cur;
         const bool have_nx = ahead.next(p, nx);
         if (have_nx && producer_q<D>(p, sm, nx, j + 1, pol))
             q_issued = j + 2;
         const int32_t *trow = p.table + (int64_t)it.s * p.table_stride;
-        if (p.P % TK != 0) {
-            // Any page size: a tile of TK positions may straddle pages, and is
-            // filled by one bulk copy per page piece (its rows land in order).
-            // The page walk moves forward piece by piece; the next page id is
-            // read one page ahead.  A piece on a page outside the pool is not
-            // read: its bytes are released with complete_tx (and flagged).
+        if (quads) {
+            // Any page size: a tile of TK positions may straddle pages.  The
+            // copy engine's cost is per copy (about 5 million copies a second
+            // per SM, whatever their size up to a tile), so tiles are armed
+            // four at a time: the quad's stages are contiguous in each ring,
+            // and one bulk copy covers a page's run of positions across them
+            // (pages of 37: about 1.1 copies per 32 positions instead of
+            // 1.9).  Each copy adds its bytes to the quad's barrier (that of
+            // its last stage), and the quad's one arrival closes it.  The
+            // page walk moves forward piece by piece; the next page id is read
+            // one page ahead.  A piece on a page outside the pool is not read
+            // (and flagged).
             int lp = it.key0 / p.P;
             int page_end = (lp + 1) * p.P;
             int32_t page = __ldg(trow + lp);
             int32_t page_nx = page_end < it.key1 ? __ldg(trow + lp + 1) : 0;
             for (int t0 = it.key0; t0 < it.key1 && !sm.abort_flag; t0 += TK, ++T) {
                 const int stage = T % NSTAGE;
+                if ((int)(T >> 2) != quad) {
+                    if (quad >= 0) {
+                        flush();
+                        mbar_arrive(&sm.full[(quad * 4 + 3) % NSTAGE]);
+                    }
+                    quad = (int)(T >> 2);
+                }
                 if (!wait_or_abort(sm, &sm.empty[stage], ((T / NSTAGE) & 1u) ^ 1u, p.flags, kWaitEmpty))
                     break;
                 sm.stage_tile[stage] = T;
                 const int t1 = min(t0 + TK, it.key1);
-                mbar_arrive_expect_tx(&sm.full[stage], 2u * static_cast<uint32_t>(t1 - t0) * D * 2u);
                 for (int pos = t0; pos < t1;) {
                     const int n = min(page_end, t1) - pos;
-                    const uint32_t nb = static_cast<uint32_t>(n) * D * 2u;
-                    if (page >= 0 && page < p.n_pages) {
-                        const size_t off =
-                            (((size_t)page * p.Hkv + it.kh) * p.P + (pos - (page_end - p.P))) * D;
-                        bulk_g2s(sm.kv[stage][0] + (pos - t0) * D * 2, p.k_pool + off, nb,
-                                 &sm.full[stage], pol);
-                        bulk_g2s(sm.kv[stage][1] + (pos - t0) * D * 2, p.v_pool + off, nb,
-                                 &sm.full[stage], pol);
+                    const int row = stage * TK + (pos - t0);
+                    // the pending run goes on if the source rows and the ring
+                    // rows both continue it
+                    if (pc_n > 0 && pc_page == page && pc_kh == it.kh && pc_pos + pc_n == pos &&
+                        pc_row + pc_n == row) {
+                        pc_n += n;
                     } else {
-                        set_flag(p.flags, kDevBadPage);
-                        mbar_complete_tx(&sm.full[stage], 2u * nb);
+                        flush();
+                        pc_n = n;
+                        pc_pos = pos;
+                        pc_row = row;
+                        pc_page = page;
+                        pc_kh = it.kh;
+                        pc_off = pos - (page_end - p.P);
                     }
                     pos += n;
                     if (pos == page_end) {
@@ -264,6 +316,23 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
                             page_nx = __ldg(trow + lp + 1);
                     }
                 }
+            }
+            // The segment's last quad closes here and the next segment starts
+            // a quad of its own: a quad never waits on a later segment, so no
+            // consumer can be held on a tile whose quad the producer closes
+            // only after a wait (the next query copy) that needs that
+            // consumer.  The skipped slots keep their empty barriers' phases
+            // in step: the producer releases them itself.
+            if (quad >= 0) {
+                flush();
+                mbar_arrive(&sm.full[(quad * 4 + 3) % NSTAGE]);
+                quad = -1;
+            }
+            for (; (T & 3u) != 0u; ++T) {
+                const int stage = T % NSTAGE;
+                if (!wait_or_abort(sm, &sm.empty[stage], ((T / NSTAGE) & 1u) ^ 1u, p.flags, kWaitEmpty))
+                    break;
+                mbar_arrive(&sm.empty[stage]);
             }
             have = have_nx;
             it = nx;
@@ -294,8 +363,8 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
                 if (page_ok) {
                     const size_t off = base + (size_t)(t0 - lp * p.P) * D;
                     mbar_arrive_expect_tx(&sm.full[stage], 2u * bytes);
-                    bulk_g2s(sm.kv[stage][0], p.k_pool + off, bytes, &sm.full[stage], pol);
-                    bulk_g2s(sm.kv[stage][1], p.v_pool + off, bytes, &sm.full[stage], pol);
+                    bulk_g2s(sm.kring[stage], p.k_pool + off, bytes, &sm.full[stage], pol);
+                    bulk_g2s(sm.vring[stage], p.v_pool + off, bytes, &sm.full[stage], pol);
                 } else {
                     mbar_arrive(&sm.full[stage]);
                 }
@@ -313,7 +382,9 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
         const uint32_t n = T < (uint32_t)NSTAGE ? T : (uint32_t)NSTAGE;
         for (uint32_t k = 1; k <= n; ++k) {
             const uint32_t t = T - k;
-            (void)mbar_wait(&sm.full[t % NSTAGE], (t / NSTAGE) & 1u, sm.wait_limit);
+            // (quads complete on the barrier of their last stage)
+            const uint32_t b = quads ? ((t | 3u) % NSTAGE) : (t % NSTAGE);
+            (void)mbar_wait(&sm.full[b], (t / NSTAGE) & 1u, sm.wait_limit);
         }
         for (uint32_t k = 1; k <= 2 && k <= q_issued; ++k) {
             const uint32_t jj = q_issued - k;  // the last two query copies started
@@ -355,6 +426,7 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
     const int grp = lane / LG;
     const int li = lane % LG;
     const float NEG_INF = -__int_as_float(0x7f800000);
+    const bool quads = p.P % TK != 0;
 
     SegCursor cur;
     cur.init(p, sm.range);
@@ -417,14 +489,16 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
             const int stage = T % NSTAGE;
             // the warp takes one decision: a lane whose wait ran out makes
             // every lane skip the tile (the CTA is winding down then)
+            // (tiles assembled from page pieces complete per quad of stages)
+            const int fs = quads ? (stage | 3) : stage;
             const bool ok = __all_sync(
                 0xffffffffu, wait_tag<D>(sm, stage, T, p.flags) &&
-                                 wait_or_abort(sm, &sm.full[stage], (T / NSTAGE) & 1u, p.flags,
+                                 wait_or_abort(sm, &sm.full[fs], (T / NSTAGE) & 1u, p.flags,
                                                kWaitFull));
             if (!ok)
                 continue;
-            const uint8_t *Ks = sm.kv[stage][0];
-            const uint8_t *Vs = sm.kv[stage][1];
+            const uint8_t *Ks = sm.kring[stage];
+            const uint8_t *Vs = sm.vring[stage];
             const int tpos = it.key0 + t * TK;
             const int nk = min(TK, it.key1 - tpos);
 
@@ -573,6 +647,8 @@ __device__ __forceinline__ void simt_consumer(const AttnParams &p, SimtSmem<D> &
                 mbar_arrive(&sm.empty[stage]);
         }
         T0 += ntiles;
+        if (quads)  // each segment's tiles start a quad (as the producer arms them)
+            T0 = (T0 + 3u) & ~3u;
 
         // --- park this warp's state; the last warp in combines -------------
         float l_row[kR];
