@@ -17,10 +17,16 @@ def small_workload(d, G, P, W, Hkv=2, seed=100, sigma=1.0):
 
 
 def run_parity(w, lens, rows, table=None, n_pages=None):
+    import verify_paged_gqa_b200 as tf
     case = synth.make_case(w, lens=lens, rows=rows, table=table, n_pages=n_pages)
     dc = DeviceCase(case)
-    out = dc.attend()
+    ws = dc.workspace(rows)
+    out = dc.attend(ws=ws)
     torch.cuda.synchronize()
+    # a clean call: no timeout, no bad length or page (a wait that ran out
+    # leaves rows unwritten, which the comparison below would also catch)
+    status = tf.tf_workspace_status(ws)
+    assert status == 0, hex(status)
     ref = oracle.attend(case.q, case.k_lin, case.v_lin, case.lens, rows, w.group, w.scale,
                         threads=8)
     assert torch.isfinite(out).all()
@@ -227,6 +233,26 @@ def test_split_many_short_streams():
     lens = [int(x) for x in rng.integers(8, 700, size=60)] + [5000, 8, 1]
     w = small_workload(128, 8, 512, 1, Hkv=2, seed=9201)
     run_parity(w, lens, 1)
+
+
+@pytest.mark.parametrize("d,top", [(128, 700), (512, 300)])
+def test_page37_many_short_segments(d, top):
+    """Decode blocks of 4 rows over pages of 37 on the CUDA-core kernel, which
+    arms straddling tiles four ring stages at a time and starts every segment
+    on a fresh quad: many short streams (segments of 1 to a few tiles, quads
+    with unused slots, tile ends on and beside page ends) match the oracle,
+    twice byte for byte, and the same streams with pages laid out in order
+    give the same bytes."""
+    rng = np.random.default_rng(9400 + d)
+    edges = [1, 7, 8, 9, 31, 32, 33, 36, 37, 38, 74, 127, 128, 129]
+    lens = [int(x) for x in rng.integers(1, top, size=40)] + edges
+    w = small_workload(d, 4, 37, 1, Hkv=2, seed=9401 + d)
+    case, dc, out = run_parity(w, lens, 1)
+    again = dc.attend()
+    assert torch.equal(out, again)
+    table, n_pages = synth.identity_table(case.lens, w.page_size)
+    inorder = DeviceCase(case, table=table, n_pages=n_pages).attend()
+    assert torch.equal(out, inorder)
 
 
 def test_split_skips_out_of_range_stream():

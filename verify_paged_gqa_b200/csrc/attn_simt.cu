@@ -322,17 +322,26 @@ __device__ __forceinline__ void simt_producer(const AttnParams &p, SimtSmem<D> &
             // consumer can be held on a tile whose quad the producer closes
             // only after a wait (the next query copy) that needs that
             // consumer.  The skipped slots keep their empty barriers' phases
-            // in step: the producer releases them itself.
+            // in step: the producer releases them itself.  It first waits for
+            // their previous tiles' releases and only then closes the quad: a
+            // quad closes once every consumer of its slots' previous round is
+            // past its wait on the quad's barrier, or that barrier could move
+            // a phase further before such a consumer looks at it.
+            const uint32_t T_end = T;
+            bool skipped_ok = true;
+            for (uint32_t Ts = T_end; (Ts & 3u) != 0u; ++Ts) {
+                const int stage = Ts % NSTAGE;
+                skipped_ok = skipped_ok && wait_or_abort(sm, &sm.empty[stage],
+                                                         ((Ts / NSTAGE) & 1u) ^ 1u, p.flags, kWaitEmpty);
+            }
             if (quad >= 0) {
                 flush();
                 mbar_arrive(&sm.full[(quad * 4 + 3) % NSTAGE]);
                 quad = -1;
             }
             for (; (T & 3u) != 0u; ++T) {
-                const int stage = T % NSTAGE;
-                if (!wait_or_abort(sm, &sm.empty[stage], ((T / NSTAGE) & 1u) ^ 1u, p.flags, kWaitEmpty))
-                    break;
-                mbar_arrive(&sm.empty[stage]);
+                if (skipped_ok)
+                    mbar_arrive(&sm.empty[T % NSTAGE]);
             }
             have = have_nx;
             it = nx;
