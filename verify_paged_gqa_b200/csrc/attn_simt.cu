@@ -58,12 +58,16 @@ template <int D>
 struct SimtCfg;
 // Registers are split per SM sub-partition: with 9 warps one sub-partition
 // holds 3 warps (at most 168 registers each), with 8 warps 2 (255 each).
+// Seven consumers (8 warps with the producer) measured faster than eight at
+// head dim 128: decode 12 x 40,960 in pages of 37 3,745 against 3,442 GB/s,
+// 64 x 2,048 5,576 against 5,160 -- the producer lane no longer shares a
+// sub-partition with two busy consumer warps.
 template <>
 struct SimtCfg<128> {
     static constexpr int TK = 32;      // positions per tile
     static constexpr int LG = 8;       // lanes sharing one key's dot product
     static constexpr int NSTAGE = 12;  // ring depth (16 KB per stage)
-    static constexpr int NCW = 8;      // consumer warps
+    static constexpr int NCW = 7;      // consumer warps
 };
 template <>
 struct SimtCfg<512> {
